@@ -1,0 +1,350 @@
+// C ABI of libsla2.so (declared in include/sla2.h): argument checks, the
+// workspace layout, TMA descriptors and the launch sequence of the forward
+// pass. Nothing here computes on the host; every step runs in the kernels.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sla2.h"
+#include "device.cuh"
+#include "kernels.cuh"
+
+using namespace sla2;
+
+namespace {
+
+constexpr unsigned long long DEFAULT_BUDGET_NS = 2000000000ull;   // 2 s per device wait
+
+unsigned long long g_budget_ns = DEFAULT_BUDGET_NS;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int topk_count(int nk, float frac) {
+  if (!(frac > 0.f) || !(frac <= 1.f) || nk < 1) return 0;
+  long long k = (long long)std::floor((double)frac * (double)nk + 1e-3);
+  if (k < 1) k = 1;
+  if (k > nk) k = nk;
+  return (int)k;
+}
+
+sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
+  if (!d) return SLA2_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->N < 1 || d->d < 1) return SLA2_ERR_INVALID_ARG;
+  if (!(frac > 0.f) || !(frac <= 1.f)) return SLA2_ERR_INVALID_ARG;
+  if (d->quantize != 0 && d->quantize != 1) return SLA2_ERR_INVALID_ARG;
+  if (d->out_dtype != 0 && d->out_dtype != 1) return SLA2_ERR_INVALID_ARG;
+  if (d->N % BQ != 0 || (d->d != 64 && d->d != 128)) return SLA2_ERR_UNSUPPORTED;
+  const long long BH = (long long)d->B * d->H;
+  if (BH * d->N > 0x7fffffffLL || BH * (d->N / BKB) * d->d > 0x7fffffffLL) return SLA2_ERR_UNSUPPORTED;
+  if (d->N / BKB > scores_topk_max_nk()) return SLA2_ERR_UNSUPPORTED;
+  s->BH = (int)BH;
+  s->N = d->N;
+  s->d = d->d;
+  s->nq = d->N / BQ;
+  s->nk = d->N / BKB;
+  s->k = topk_count(s->nk, frac);
+  return SLA2_OK;
+}
+
+// Workspace regions (each 256-byte aligned).
+struct Layout {
+  size_t qbar, ksum, c64, c32, A, Bk, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
+      os, total;
+};
+
+Layout make_layout(const Shape& s, int quant) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t BH = s.BH, N = s.N, d = s.d, nq = s.nq, nk = s.nk, k = s.k;
+  const size_t G = linear_chunks(s.nk);
+  L.qbar = take(BH * nq * d * 4);
+  L.ksum = take(BH * nk * d * 8);
+  L.c64 = take(BH * d * 8);
+  L.c32 = take(BH * d * 4);
+  L.A = take(BH * nq * d * 4);
+  L.Bk = take(BH * nk * d * 4);
+  L.mask = take(BH * nq * nk);
+  L.idx = take(BH * nq * k * 4);
+  L.qhat = take(quant ? BH * N * d : 0);
+  L.sq = take(BH * nq * 4);
+  L.vamax = take(BH * d * 4);
+  L.khat = take(quant ? BH * N * d : 0);
+  L.sk = take(BH * nk * 4);
+  L.vhatT = take(BH * nk * d * BKB * (quant ? 1 : 2));
+  L.sv = take(BH * d * 4);
+  L.h = take(BH * nk * d * d * 4);
+  L.z = take(BH * nk * d * 4);
+  L.hpart = take(BH * G * d * d * 4);
+  L.zpart = take(BH * G * d * 4);
+  L.Htot = take(BH * d * d * 4);
+  L.Ztot = take(BH * d * 4);
+  L.os = take(BH * N * d * 4);
+  L.total = off;
+  return L;
+}
+
+template <class T>
+T* at(const sla2_desc* d, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(d->workspace) + off);
+}
+
+// ---- TMA descriptors (driver entry point fetched once through the runtime)
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D row-major map: `rows` rows of `cols` elements, box = box_cols x box_rows.
+bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, uint64_t cols, uint64_t rows,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (cuuint64_t)esz};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+sla2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA2_OK : SLA2_ERR_CUDA; }
+
+#define SLA2_TRY(expr)                                   \
+  do {                                                   \
+    cudaError_t _e = (expr);                             \
+    if (_e != cudaSuccess) return SLA2_ERR_CUDA;         \
+  } while (0)
+
+sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
+                       const void* v, const float* wq, const float* wk, uint8_t* mask, int32_t* idx, int quant,
+                       cudaStream_t st) {
+  if (quant) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
+  SLA2_TRY(launch_pool(s, q, k, quant ? v : nullptr, at<float>(d, L.qbar), at<double>(d, L.ksum),
+                       quant ? at<int8_t>(d, L.qhat) : nullptr, at<float>(d, L.sq),
+                       quant ? at<unsigned>(d, L.vamax) : nullptr, st));
+  SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), st));
+  SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<double>(d, L.ksum), at<double>(d, L.c64), wq, wk,
+                       at<float>(d, L.A), at<float>(d, L.Bk), st));
+  SLA2_TRY(launch_scores_topk(s, at<float>(d, L.A), at<float>(d, L.Bk), mask, idx, d->dbg_scores, st));
+  return SLA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sla2_status_string(sla2_status s) {
+  switch (s) {
+    case SLA2_OK: return "ok";
+    case SLA2_ERR_INVALID_ARG: return "invalid argument";
+    case SLA2_ERR_UNSUPPORTED: return "unsupported shape (N % 128 != 0, d not in {64,128}, or too large)";
+    case SLA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SLA2_ERR_CUDA: return "CUDA error";
+    case SLA2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+  }
+  return "unknown status";
+}
+
+int sla2_topk_count(int nk, float topk_frac) { return topk_count(nk, topk_frac); }
+
+size_t sla2_workspace_size(const sla2_desc* desc, float topk_frac) {
+  Shape s;
+  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
+  return make_layout(s, desc->quantize).total;
+}
+
+// Test knob: the budget (ns) of every bounded device wait in later launches;
+// 0 restores the default (declared in include/sla2_test.h).
+void sla2_set_wait_budget_ns(unsigned long long ns) { g_budget_ns = ns ? ns : DEFAULT_BUDGET_NS; }
+
+sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
+                        const float* proj_k, float topk_frac, uint8_t* mask_out, int32_t* idx_out,
+                        float* colmean_out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !proj_q || !proj_k || !mask_out || !idx_out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  r = run_router(desc, s, L, q, k, nullptr, proj_q, proj_k, mask_out, idx_out, 0, st);
+  if (r != SLA2_OK) return r;
+  if (colmean_out)
+    SLA2_TRY(cudaMemcpyAsync(colmean_out, at<float>(desc, L.c32), (size_t)s.BH * s.d * 4, cudaMemcpyDeviceToDevice, st));
+  return SLA2_OK;
+}
+
+sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v, const float* colmean,
+                              float* h_out, float* z_out, float* Htot_out, float* Ztot_out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, 1.f, &s);
+  if (r != SLA2_OK) return r;
+  if (!k || !v || !colmean || !h_out || !z_out || !Htot_out || !Ztot_out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(h_out) || !aligned16(Htot_out)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LinearOut o{};
+  o.h = h_out;
+  o.z = z_out;
+  o.hpart = at<float>(desc, L.hpart);
+  o.zpart = at<float>(desc, L.zpart);
+  o.quant = 0;
+  SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, Htot_out, Ztot_out, st));
+  return SLA2_OK;
+}
+
+sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v, const float* proj_q,
+                         const float* proj_k, const float* alpha, float topk_frac, void* out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj_q) || !aligned16(proj_k) ||
+      !aligned16(out))
+    return SLA2_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return SLA2_ERR_INVALID_ARG;
+  const int quant = desc->quantize;
+  const Layout L = make_layout(s, quant);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  if (!get_encode()) return SLA2_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> cudaError_t {
+    if (!desc->stage_events) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(desc->stage_events[i]), st);
+  };
+  if (desc->status) SLA2_TRY(cudaMemsetAsync(desc->status, 0, sizeof(unsigned), st));
+  SLA2_TRY(mark(0));
+
+  uint8_t* mask = at<uint8_t>(desc, L.mask);
+  int32_t* idx = at<int32_t>(desc, L.idx);
+  r = run_router(desc, s, L, q, k, v, proj_q, proj_k, mask, idx, quant, st);
+  if (r != SLA2_OK) return r;
+  SLA2_TRY(mark(1));
+
+  LinearOut o{};
+  o.h = at<float>(desc, L.h);
+  o.z = at<float>(desc, L.z);
+  o.hpart = at<float>(desc, L.hpart);
+  o.zpart = at<float>(desc, L.zpart);
+  o.khat = quant ? at<int8_t>(desc, L.khat) : nullptr;
+  o.sk = at<float>(desc, L.sk);
+  o.vhatT = at<void>(desc, L.vhatT);
+  o.sv = at<float>(desc, L.sv);
+  o.vamax = at<unsigned>(desc, L.vamax);
+  o.quant = quant;
+  SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, at<float>(desc, L.Htot), at<float>(desc, L.Ztot), st));
+  SLA2_TRY(mark(2));
+
+  // sparse branch: tensor maps over the (quantised) operands
+  CUtensorMap tq, tk, tv;
+  const uint64_t rows = (uint64_t)s.BH * s.N, vrows = (uint64_t)s.BH * s.nk * s.d;
+  bool okm;
+  if (quant) {
+    const CUtensorMapSwizzle sw = s.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    okm = make_map(&tq, at<void>(desc, L.qhat), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, rows, s.d, BQ, sw) &&
+          make_map(&tk, at<void>(desc, L.khat), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, rows, s.d, BKB, sw) &&
+          make_map(&tv, at<void>(desc, L.vhatT), CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, BKB, vrows, BKB, s.d,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
+  } else {
+    okm = make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B) &&
+          make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BKB, CU_TENSOR_MAP_SWIZZLE_128B) &&
+          make_map(&tv, at<void>(desc, L.vhatT), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BKB, vrows, BKB, s.d,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  if (!okm) return SLA2_ERR_CUDA;
+  float* os = desc->dbg_os ? desc->dbg_os : at<float>(desc, L.os);
+  SparseArgs sa{idx, at<float>(desc, L.sq), at<float>(desc, L.sk), at<float>(desc, L.sv), os, desc->status, g_budget_ns};
+  SLA2_TRY(launch_sparse(s, quant, tq, tk, tv, sa, st));
+  SLA2_TRY(mark(3));
+
+  EpilogueArgs ea{};
+  ea.q = q;
+  ea.Htot = at<float>(desc, L.Htot);
+  ea.Ztot = at<float>(desc, L.Ztot);
+  ea.h = o.h;
+  ea.z = o.z;
+  ea.idx = idx;
+  ea.os = os;
+  ea.alpha = alpha;
+  ea.H = desc->H;
+  ea.out = out;
+  ea.out_f32 = desc->out_dtype;
+  ea.ol_dbg = desc->dbg_ol;
+  SLA2_TRY(launch_epilogue(s, ea, st));
+  SLA2_TRY(mark(4));
+
+  // debug exports
+  auto cp = [&](void* dst, size_t off, size_t bytes) -> cudaError_t {
+    if (!dst) return cudaSuccess;
+    return cudaMemcpyAsync(dst, at<uint8_t>(desc, off), bytes, cudaMemcpyDeviceToDevice, st);
+  };
+  const size_t BH = s.BH;
+  SLA2_TRY(cp(desc->dbg_mask, L.mask, BH * s.nq * s.nk));
+  SLA2_TRY(cp(desc->dbg_idx, L.idx, BH * s.nq * s.k * 4));
+  if (quant) {
+    SLA2_TRY(cp(desc->dbg_qhat, L.qhat, BH * s.N * s.d));
+    SLA2_TRY(cp(desc->dbg_khat, L.khat, BH * s.N * s.d));
+    SLA2_TRY(cp(desc->dbg_vhat, L.vhatT, BH * s.nk * s.d * BKB));
+    SLA2_TRY(cp(desc->dbg_qscale, L.sq, BH * s.nq * 4));
+    SLA2_TRY(cp(desc->dbg_kscale, L.sk, BH * s.nk * 4));
+    SLA2_TRY(cp(desc->dbg_vscale, L.sv, BH * s.d * 4));
+  }
+  return SLA2_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded device wait (declared in include/sla2_test.h): one
+// warp waits on an mbarrier that nothing arrives on; after `budget_ns` the
+// wait gives up, writes SLA2_ERR_DEVICE_TIMEOUT into *status and the kernel
+// returns normally.
+namespace {
+__global__ void timeout_probe_kernel(unsigned* status, unsigned long long budget_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sla2::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sla2::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sla2::mbar_wait(&bar, 0, &abort_flag, status, budget_ns);
+}
+}  // namespace
+
+extern "C" sla2_status sla2_selftest_timeout(unsigned* status, unsigned long long budget_ns, void* stream) {
+  if (!status || budget_ns == 0 || budget_ns > 10000000000ull) return SLA2_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(cudaMemsetAsync(status, 0, sizeof(unsigned), st));
+  timeout_probe_kernel<<<1, 32, 0, st>>>(status, budget_ns);
+  return cuda_status(cudaGetLastError());
+}

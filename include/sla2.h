@@ -1,0 +1,136 @@
+/*
+ * sla2.h -- C ABI of libsla2.so: the SLA2 sparse-linear attention inference
+ * forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources: the SLA2 summary page at paper.rainbus.top, first
+ * paragraph, steps 1-4; the SLA2 detail page at zhaifeiyue.github.io, §3
+ * flowchart, §4 symbol table, §7 implementation notes):
+ *
+ *   K_s  = K - colmean(K)                                    (detail §7, note 1)
+ *   Qbar = mean-pool(Q, 128 tokens), Kbar = mean-pool(K_s, 64 tokens)
+ *   s    = (Qbar Wq)(Kbar Wk)^T / sqrt(d); M_c = hard top-k per row      (step 1)
+ *   O_s  = softmax attention over the selected blocks, INT8 Q/K, FP8 P/V (step 2)
+ *   O_l  = phi(Q_i) H_i / (phi(Q_i) Z_i), H_i, Z_i over unselected blocks (step 3)
+ *   O    = alpha * O_s + (1 - alpha) * O_l                               (step 4)
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or synchronises. Scratch memory is the caller's
+ *     workspace (see sla2_workspace_size).
+ *   - Q, K, V, out: contiguous [B][H][N][d]; Q/K/V bf16; out bf16 or fp32.
+ *     proj_q, proj_k: fp32 [H][d][d], applied as y = x W (row vector times W,
+ *     W stored [d_in][d_out]). alpha: fp32 [H][N/128], shared over the batch,
+ *     used as given (expected in [0, 1]).
+ *   - Shapes: N % 128 == 0, d in {64, 128}, B, H >= 1. Every base pointer must
+ *     be 16-byte aligned. out must not alias an input.
+ *   - k (key blocks kept per query block) = clamp(floor(frac * nk + 1e-3), 1, nk)
+ *     with nk = N / 64; frac must lie in (0, 1].
+ *   - Calls enqueue on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and return. SLA2_OK means "arguments valid and kernels enqueued".
+ *     Arguments are checked before any launch; on an argument error nothing is
+ *     written. Launch failures return SLA2_ERR_CUDA.
+ *   - A workspace may be reused by back-to-back calls on one stream; calls that
+ *     may run concurrently need separate workspaces.
+ *   - Device-side waits are bounded; a wait that runs out writes a nonzero code
+ *     into the optional status word (desc.status) and the kernel returns.
+ */
+#ifndef SLA2_H
+#define SLA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA2_OK = 0,
+  SLA2_ERR_INVALID_ARG = 1,    /* NULL pointer, bad size, frac outside (0,1], misalignment */
+  SLA2_ERR_UNSUPPORTED = 2,    /* N % 128 != 0 or d not in {64, 128} */
+  SLA2_ERR_WORKSPACE = 3,      /* workspace NULL or smaller than sla2_workspace_size() */
+  SLA2_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  SLA2_ERR_DEVICE_TIMEOUT = 5  /* reported through the status word, after a sync */
+} sla2_status;
+
+/* Problem description shared by all entry points. */
+typedef struct {
+  int B, H, N, d;
+  int quantize;        /* 1: INT8 Q/K + FP8 e4m3 P/V sparse branch (default);
+                          0: bf16 tensor-core sparse branch (no quantisation)   */
+  int out_dtype;       /* 0: bf16 output, 1: fp32 output                        */
+  void* workspace;     /* device scratch, >= sla2_workspace_size() bytes,
+                          256-byte aligned                                      */
+  size_t workspace_bytes;
+  unsigned int* status;/* optional device word; set to 0 at each call and to a
+                          nonzero SLA2_ERR_DEVICE_TIMEOUT code if a bounded
+                          device wait ran out                                   */
+  /* Optional debug exports (NULL = not written), all device pointers:        */
+  float* dbg_scores;   /* router logits s, fp32 [B][H][N/128][N/64]            */
+  float* dbg_os;       /* sparse branch O_s, fp32 [B][H][N][d]                 */
+  float* dbg_ol;       /* linear branch O_l, fp32 [B][H][N][d]                 */
+  int8_t* dbg_qhat;    /* INT8 Q-hat [B][H][N][d]  (quantize = 1 only)          */
+  int8_t* dbg_khat;    /* INT8 K-hat of K_s [B][H][N][d]                        */
+  uint8_t* dbg_vhat;   /* e4m3 V-hat codes in the layout the sparse kernel reads:
+                          per key block, channel-major [B][H][N/64][d][64]     */
+  float* dbg_qscale;   /* s_q [B][H][N/128]                                     */
+  float* dbg_kscale;   /* s_k [B][H][N/64]                                      */
+  float* dbg_vscale;   /* s_v [B][H][d]                                         */
+  uint8_t* dbg_mask;   /* M_c [B][H][N/128][N/64]                               */
+  int32_t* dbg_idx;    /* selected block indices, ascending, [B][H][N/128][k]   */
+  /* Optional timing hooks: NULL, or an array of SLA2_STAGE_EVENTS cudaEvent_t
+     that sla2_forward records on `stream` at the stage boundaries
+     [start, router done, linear state done, sparse branch done, end].       */
+  void* const* stage_events;
+} sla2_desc;
+
+#define SLA2_STAGE_EVENTS 5
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sla2_status_string(sla2_status s);
+
+/* k for a given key-block count and fraction (see conventions); 0 if frac is
+ * outside (0, 1] or nk < 1. Host-only, no CUDA call. */
+int sla2_topk_count(int nk, float topk_frac);
+
+/* Bytes of device workspace sla2_forward needs for this description and
+ * fraction; 0 if the description is invalid. Host-only, no CUDA call. */
+size_t sla2_workspace_size(const sla2_desc* desc, float topk_frac);
+
+/* Steps 1 (and K smoothing) only: the learnable router.
+ *   q, k      : bf16 [B][H][N][d]
+ *   proj_q/k  : fp32 [H][d][d]
+ *   mask_out  : uint8 [B][H][N/128][N/64], M_c (1 = selected)
+ *   idx_out   : int32 [B][H][N/128][k], selected key blocks in ascending order
+ *   colmean_out: fp32 [B][H][d] (the K smoothing mean, rounded to fp32) or NULL
+ * Uses desc->workspace (sla2_workspace_size bytes suffice); desc->dbg_scores
+ * receives the fp32 logits when non-NULL. Top-k ties go to the lower index.
+ * (Summary page, step 1; detail page §3 "Learnable Router".) */
+sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k,
+                        const float* proj_q, const float* proj_k, float topk_frac,
+                        uint8_t* mask_out, int32_t* idx_out, float* colmean_out,
+                        void* stream);
+
+/* Step 3's per-key-block linear-attention state (detail page §7, note 2:
+ * h_j precomputed per key block, then accumulated):
+ *   phi(x) = softmax over the d features; K_s = K - colmean (fp32)
+ *   h_out    : fp32 [B][H][N/64][d][d], h_j = phi(K_s,j)^T V_j
+ *   z_out    : fp32 [B][H][N/64][d],    z_j = column sums of phi(K_s,j)
+ *   Htot_out : fp32 [B][H][d][d] = sum_j h_j;  Ztot_out: fp32 [B][H][d]
+ *   colmean  : fp32 [B][H][d] as returned by sla2_router.
+ * Uses desc->workspace for the partial sums. */
+sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v,
+                              const float* colmean, float* h_out, float* z_out,
+                              float* Htot_out, float* Ztot_out, void* stream);
+
+/* The whole forward pass (steps 1-4): out = alpha O_s + (1 - alpha) O_l.
+ *   out : bf16 or fp32 (desc->out_dtype) [B][H][N][d]
+ * All intermediates live in desc->workspace; optional debug exports in desc. */
+sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v,
+                         const float* proj_q, const float* proj_k, const float* alpha,
+                         float topk_frac, void* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLA2_H */
