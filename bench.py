@@ -57,11 +57,12 @@ def work_model(w, k):
         "effective_ops": 4 * B * H * N * N * d,
         # router: read Q, K, V (bf16), write Q-hat (int8)
         "router_bytes": 2 * E * 3 + E,
-        # linear state: read K, V (bf16), write K-hat, V-hat^T (8-bit), h_j, z_j (fp32)
-        "linear_bytes": 2 * E * 2 + 2 * E + BH * nk * d * d * 4 + BH * nk * d * 4,
-        # epilogue: read Q (bf16), O_s (fp32), write out (bf16); the h_j gather is L2 traffic
-        "epilogue_bytes": 2 * E + 4 * E + 2 * E,
-        "gather_bytes": BH * nq * k * d * d * 4,
+        # linear state: read K, V (bf16), write K-hat, V-hat^T (8-bit), h_j^T (bf16), z_j (fp32)
+        "linear_bytes": 2 * E * 2 + 2 * E + BH * nk * d * d * 2 + BH * nk * d * 4,
+        # epilogue: read Q (bf16), O_s (fp32), h_j^T once (bf16), write out (bf16); the
+        # repeated h_j^T gather (k per query block) is L2 traffic, reported separately
+        "epilogue_bytes": 2 * E + 4 * E + 2 * E + BH * nk * d * d * 2,
+        "gather_bytes": BH * nq * k * d * d * 2,
     }
 
 

@@ -53,7 +53,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 
 // Workspace regions (each 256-byte aligned).
 struct Layout {
-  size_t qbar, ksum, c64, c32, A, Bk, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
+  size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
       os, total;
 };
 
@@ -66,13 +66,15 @@ Layout make_layout(const Shape& s, int quant) {
     return o;
   };
   const size_t BH = s.BH, N = s.N, d = s.d, nq = s.nq, nk = s.nk, k = s.k;
-  const size_t G = linear_chunks(s.nk);
+  const size_t G = linear_chunks(s.BH, s.nk);
   L.qbar = take(BH * nq * d * 4);
   L.ksum = take(BH * nk * d * 8);
   L.c64 = take(BH * d * 8);
   L.c32 = take(BH * d * 4);
+  L.kbs = take(BH * nk * d * 4);
   L.A = take(BH * nq * d * 4);
   L.Bk = take(BH * nk * d * 4);
+  L.scores = take(BH * nq * nk * 4);
   L.mask = take(BH * nq * nk);
   L.idx = take(BH * nq * k * 4);
   L.qhat = take(quant ? BH * N * d : 0);
@@ -82,7 +84,7 @@ Layout make_layout(const Shape& s, int quant) {
   L.sk = take(BH * nk * 4);
   L.vhatT = take(BH * nk * d * BKB * (quant ? 1 : 2));
   L.sv = take(BH * d * 4);
-  L.h = take(BH * nk * d * d * 4);
+  L.h = take(BH * nk * d * d * 2);   // bf16 h_j^T
   L.z = take(BH * nk * d * 4);
   L.hpart = take(BH * G * d * d * 4);
   L.zpart = take(BH * G * d * 4);
@@ -125,6 +127,20 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, 
   return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+bool sla2::make_tmap_2d(CUtensorMap* m, const void* ptr, int esz, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                        uint32_t box_rows, int swizzle_bytes) {
+  if (!get_encode()) return false;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return make_map(m, ptr, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, esz, cols,
+                  rows, box_cols, box_rows, sw);
+}
+
+namespace {
+
 sla2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA2_OK : SLA2_ERR_CUDA; }
 
 #define SLA2_TRY(expr)                                   \
@@ -140,10 +156,13 @@ sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, cons
   SLA2_TRY(launch_pool(s, q, k, quant ? v : nullptr, at<float>(d, L.qbar), at<double>(d, L.ksum),
                        quant ? at<int8_t>(d, L.qhat) : nullptr, at<float>(d, L.sq),
                        quant ? at<unsigned>(d, L.vamax) : nullptr, st));
-  SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), st));
-  SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<double>(d, L.ksum), at<double>(d, L.c64), wq, wk,
-                       at<float>(d, L.A), at<float>(d, L.Bk), st));
-  SLA2_TRY(launch_scores_topk(s, at<float>(d, L.A), at<float>(d, L.Bk), mask, idx, d->dbg_scores, st));
+  SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), at<float>(d, L.kbs),
+                           st));
+  SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<float>(d, L.kbs), wq, wk, at<float>(d, L.A),
+                       at<float>(d, L.Bk), st));
+  float* scores = d->dbg_scores ? d->dbg_scores : at<float>(d, L.scores);
+  SLA2_TRY(launch_scores(s, at<float>(d, L.A), at<float>(d, L.Bk), scores, st));
+  SLA2_TRY(launch_topk(s, scores, mask, idx, st));
   return SLA2_OK;
 }
 
@@ -209,10 +228,13 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   LinearOut o{};
   o.h = h_out;
+  o.h_mode = 0;
   o.z = z_out;
   o.hpart = at<float>(desc, L.hpart);
   o.zpart = at<float>(desc, L.zpart);
   o.quant = 0;
+  o.status = desc->status;
+  o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, Htot_out, Ztot_out, st));
   return SLA2_OK;
@@ -249,7 +271,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   SLA2_TRY(mark(1));
 
   LinearOut o{};
-  o.h = at<float>(desc, L.h);
+  o.h = at<void>(desc, L.h);
+  o.h_mode = 1;
   o.z = at<float>(desc, L.z);
   o.hpart = at<float>(desc, L.hpart);
   o.zpart = at<float>(desc, L.zpart);
@@ -259,6 +282,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   o.sv = at<float>(desc, L.sv);
   o.vamax = at<unsigned>(desc, L.vamax);
   o.quant = quant;
+  o.status = desc->status;
+  o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, at<float>(desc, L.Htot), at<float>(desc, L.Ztot), st));
   SLA2_TRY(mark(2));
@@ -289,7 +314,7 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.q = q;
   ea.Htot = at<float>(desc, L.Htot);
   ea.Ztot = at<float>(desc, L.Ztot);
-  ea.h = o.h;
+  ea.hT = at<uint16_t>(desc, L.h);
   ea.z = o.z;
   ea.idx = idx;
   ea.os = os;
@@ -298,6 +323,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.out = out;
   ea.out_f32 = desc->out_dtype;
   ea.ol_dbg = desc->dbg_ol;
+  ea.status = desc->status;
+  ea.budget_ns = g_budget_ns;
   SLA2_TRY(launch_epilogue(s, ea, st));
   SLA2_TRY(mark(4));
 

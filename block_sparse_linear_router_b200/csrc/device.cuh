@@ -148,10 +148,19 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       : "memory");
 }
 
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 // Instruction descriptor (dense, no negate, both operands K-major).
 //   bits 4-5 D format (1 = f32, 2 = s32); 7-9 A format; 10-12 B format;
 //   17-22 N >> 3; 24-28 M >> 4.
-// A/B formats: kind::i8 1 = signed int8; kind::f8f6f4 0 = e4m3; kind::f16 1 = bf16.
+// A/B formats: kind::i8 1 = signed int8; kind::f8f6f4 0 = e4m3; kind::f16 0 = fp16,
+// 1 = bf16; kind::tf32 2 = tf32 (fp32 words, low mantissa bits ignored).
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t dfmt, uint32_t afmt, uint32_t bfmt, uint32_t M, uint32_t N) {
   return (dfmt << 4) | (afmt << 7) | (bfmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
@@ -210,6 +219,18 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// fp32 -> tf32 (round to nearest, ties away), returned as an fp32 bit pattern.
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+// Byte offset of element (row, col) of a K-major fp32 operand tile stored as
+// 128-byte-swizzled slabs of 32 columns; `slab_bytes` = rows * 128.
+__device__ __forceinline__ uint32_t sw128_f32(int row, int col, int slab_bytes) {
+  const int slab = col >> 5, chunk = (col & 31) >> 2;
+  return (uint32_t)(slab * slab_bytes + row * 128 + ((chunk ^ (row & 7)) << 4) + ((col & 3) << 2));
 }
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -3,15 +3,21 @@
 // note 2: h_j precomputed per key block, then accumulated; step 2's low-bit K
 // and V).
 //
-// One CTA walks a contiguous chunk of key blocks of one head. Per key block j:
-//   K_s = fp32(K) - fp32(c)                      (K smoothing, detail §7 note 1)
-//   K-hat_j = INT8 of K_s over the 64 x d block, s_k = amax / 127
-//   V-hat_j^T = e4m3(V * 448 / amax_channel) stored channel-major [d][64]
-//   phi(K_s) = softmax over the d features (fp32, accurate expf)
-//   z_j = sum_t phi_t, h_j = phi^T V  (fp32)
-// and the chunk's partial sums of h_j, z_j, later reduced in a fixed order to
-// H_total, Z_total.
+// One CTA walks a contiguous chunk of key blocks of one head (chunks sized so
+// that all CTAs run in one wave at two CTAs per SM). Per key block j:
+//   K_s   = fp32(K) - fp32(c)                      (K smoothing, detail §7 note 1)
+//   K-hat = INT8 of K_s over the 64 x d block, s_k = amax / 127
+//   V-hat^T = e4m3(V * 448 / amax_channel), channel-major [d][64]
+//   phi   = softmax of each K_s row over the d features (fp32, accurate expf)
+//   z_j   = sum over the block's tokens of phi                   (fp32)
+//   h_j^T = V_j^T phi_j  on the tensor core: tcgen05 kind::f16 with fp16
+//           operands (V exactly, phi rounded once), fp32 accumulation in TMEM;
+//           a second TMEM accumulator sums h_j^T over the chunk (partial H^T).
+// Roles: warps 0-3 convert (TMA-staged bf16 tiles -> operands, quantised
+// copies, phi, z) and read results back from TMEM; warp 4 lane 0 issues the
+// TMA loads (two stages) and the MMAs.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "device.cuh"
 #include "kernels.cuh"
@@ -20,8 +26,25 @@ namespace sla2 {
 
 namespace {
 
-constexpr int LIN_THREADS = 256;
-constexpr int LIN_CHUNKS = 32;
+constexpr int LIN_THREADS = 160;     // 4 converter warps + 1 TMA / MMA warp
+
+template <int D>
+struct LinCfg {
+  static constexpr int SLABS = D / 64;                 // 64 bf16 = 128-byte slabs of a staged K/V tile
+  static constexpr int KV_TILE = BKB * D * 2;          // bytes of one staged bf16 K (or V) tile
+  static constexpr int STAGE = 2 * KV_TILE;            // K + V
+  static constexpr int EG = D / 8;                     // feature groups of 8 per token row
+  static constexpr int TG = 128 / EG;                  // token groups
+  static constexpr int TPT = BKB / TG;                 // tokens per converter thread
+  static constexpr int OFF_A = 2 * STAGE;              // V^T operand (MMA A: M = 128 rows, channels c < D)
+  static constexpr int OFF_B = OFF_A + 128 * 128;      // phi^T operand (MMA B: N = D rows of features e)
+  static constexpr int OFF_RED = OFF_B + D * 128;      // z partials [2][TG][D] + amax [2][4]
+  static constexpr int OFF_BAR = OFF_RED + (2 * TG * D + 8) * 4;
+  static constexpr int SMEM = OFF_BAR + 64 + 1024;
+  static constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
+  static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
+  static constexpr uint32_t COL_TOT = D;                // running partial H^T
+};
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
@@ -30,183 +53,314 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
 }
 
+__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// named barrier over the 128 converter threads (warps 0-3)
+__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 template <int D>
-__global__ void __launch_bounds__(LIN_THREADS) linear_state_kernel(
-    const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin, const float* __restrict__ c32,
-    int N, int nk, LinearOut o) {
-  constexpr int TPR = D / 8;              // threads per token row (8 channels each)
-  constexpr int RPP = LIN_THREADS / TPR;  // token rows per pass
-  constexpr int NP = BKB / RPP;           // passes over 64 tokens
-  constexpr int T = D / 16;               // h tile per thread: T x T
-  extern __shared__ float lsm[];
-  float* phi = lsm;                  // [64][D]
-  float* vs = phi + BKB * D;         // [64][D]
-  float* cs = vs + BKB * D;          // [D]
-  float* vinv = cs + D;              // [D] 448 / amax
-  float* red8 = vinv + D;            // [8]
-  const int bh = blockIdx.y, chunk = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
+__global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __grid_constant__ CUtensorMap tk,
+                                                                      const __grid_constant__ CUtensorMap tv,
+                                                                      const float* __restrict__ c32, int N, int nk,
+                                                                      LinearOut o) {
+  using C = LinCfg<D>;
+  extern __shared__ uint8_t lsm_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base + C::OFF_A;
+  uint8_t* sB = base + C::OFF_B;
+  float* zred_all = reinterpret_cast<float*>(base + C::OFF_RED);     // [2][TG][D]
+  float* ared_all = zred_all + 2 * C::TG * D;                        // [2][4]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint64_t* tma_full = bar;          // [2]
+  uint64_t* conv_done = bar + 2;
+  uint64_t* mma_done = bar + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
+  int* abort_flag = reinterpret_cast<int*>(bar + 5);        // bar + 6: drain barrier
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, chunk = blockIdx.x, G = gridDim.x;
   const int j0 = (int)((long long)chunk * nk / G), j1 = (int)((long long)(chunk + 1) * nk / G);
-  const int cg = tid % TPR, rg = tid / TPR;
-  const int ty = tid / 16, tx = tid % 16;
+  const int cnt = j1 - j0;
 
-  for (int e = tid; e < D; e += LIN_THREADS) {
-    cs[e] = c32[(size_t)bh * D + e];
-    if (o.quant == 1) {
-      const float a = __uint_as_float(o.vamax[(size_t)bh * D + e]);
-      vinv[e] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
-      if (chunk == 0) o.sv[(size_t)bh * D + e] = a > 0.f ? __fdiv_rn(a, 448.f) : 0.f;
-    }
+  if (tid == 0) {
+    mbar_init(tma_full, 1);
+    mbar_init(tma_full + 1, 1);
+    mbar_init(conv_done, 128);
+    mbar_init(mma_done, 1);
+    mbar_init(bar + 6, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  float hp[T][T];
-#pragma unroll
-  for (int a = 0; a < T; ++a)
-#pragma unroll
-    for (int b = 0; b < T; ++b) hp[a][b] = 0.f;
-  float zp = 0.f;
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  for (int j = j0; j < j1; ++j) {
-    const size_t rowbase = (size_t)bh * N + (size_t)j * BKB;
-    float x[NP][8];
-    float amax = 0.f;
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA + MMA issuer
+    if (lane == 0 && cnt > 0) {
+      auto load = [&](int n) {
+        uint8_t* stg = base + (n & 1) * C::STAGE;
+        const int row = bh * N + (j0 + n) * BKB;
+        mbar_arrive_expect_tx(tma_full + (n & 1), C::STAGE);
 #pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      const int t = p * RPP + rg;
-      const uint4 wk = __ldg(reinterpret_cast<const uint4*>(kin + (rowbase + t) * D + cg * 8));
-      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(vin + (rowbase + t) * D + cg * 8));
-      float kv[8], vv[8];
-      unpack8(wk, kv);
-      unpack8(wv, vv);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        x[p][c] = __fsub_rn(kv[c], cs[cg * 8 + c]);
-        amax = fmaxf(amax, fabsf(x[p][c]));
-        vs[t * D + cg * 8 + c] = vv[c];
-      }
-      // phi: softmax over the D features of token t (TPR consecutive lanes share the row)
-      float m = x[p][0];
-#pragma unroll
-      for (int c = 1; c < 8; ++c) m = fmaxf(m, x[p][c]);
-#pragma unroll
-      for (int off = TPR / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      float e[8], s = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        e[c] = expf(x[p][c] - m);
-        s += e[c];
-      }
-#pragma unroll
-      for (int off = TPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      const float inv = 1.f / s;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) phi[t * D + cg * 8 + c] = e[c] * inv;
-    }
-    // K-hat of the smoothed block
-    if (o.khat) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      if ((tid & 31) == 0) red8[tid >> 5] = amax;
-      __syncthreads();
-      float a = red8[0];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) a = fmaxf(a, red8[w]);
-      const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        const int t = p * RPP + rg;
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(x[p][c], inv))));
-          const int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(x[p][c + 4], inv))));
-          lo |= (uint32_t)(q0 & 0xFF) << (8 * c);
-          hi |= (uint32_t)(q1 & 0xFF) << (8 * c);
+        for (int sl = 0; sl < C::SLABS; ++sl) {
+          tma_load_2d(stg + sl * BKB * 128, &tk, tma_full + (n & 1), sl * 64, row);
+          tma_load_2d(stg + C::KV_TILE + sl * BKB * 128, &tv, tma_full + (n & 1), sl * 64, row);
         }
-        *reinterpret_cast<uint2*>(o.khat + (rowbase + t) * D + cg * 8) = make_uint2(lo, hi);
+      };
+      load(0);
+      if (cnt > 1) load(1);
+      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+      for (int n = 0; n < cnt; ++n) {
+        if (!mbar_wait(conv_done, n & 1, abort_flag, o.status, o.budget_ns)) break;
+        if (n + 2 < cnt) load(n + 2);      // stage n & 1 has been read
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < BKB / 16; ++ks) {
+          const uint64_t ad = make_sdesc(a0 + ks * 32, 1024, LAYOUT_SW128);
+          const uint64_t bd = make_sdesc(b0 + ks * 32, 1024, LAYOUT_SW128);
+          mma_f16(tmem, ad, bd, C::IDESC, ks > 0);
+          mma_f16(tmem + C::COL_TOT, ad, bd, C::IDESC, (n > 0 || ks > 0));
+        }
+        tc_commit(mma_done);
       }
-      if (tid == 0) o.sk[(size_t)bh * nk + j] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
+      if (*(volatile int*)abort_flag) {
+        // let in-flight copies land and issued MMAs finish before the CTA releases its memory
+        for (int n = (cnt > 2 ? cnt - 2 : 0); n < cnt; ++n) mbar_wait_drain(tma_full + (n & 1), (n >> 1) & 1, 20000000ull);
+        tc_commit(bar + 6);
+        mbar_wait_drain(bar + 6, 0, 20000000ull);
+      }
     }
-    __syncthreads();   // phi, vs complete
-    // V-hat^T (or the bf16 V^T copy): channel-major 64 tokens per row
-    if (o.vhatT) {
-      constexpr int HALVES = LIN_THREADS / D;      // threads per channel row
-      constexpr int TOK = BKB / HALVES;            // tokens per thread
-      const int c = tid / HALVES, part = tid % HALVES;
-      const size_t orow = ((size_t)bh * nk + j) * D + c;
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- converters (128 threads)
+    constexpr int EG = C::EG, TG = C::TG, TPT = C::TPT;
+    const int tg = tid / EG;          // token group: tokens tg*TPT .. +TPT
+    const int eg = tid % EG;          // feature / channel group: 8 columns eg*8 ..
+    const int sl = eg >> 3, ch = eg & 7;
+    float cs[8], vinv[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      cs[c] = c32[(size_t)bh * D + eg * 8 + c];
+      vinv[c] = 0.f;
       if (o.quant == 1) {
-        uint8_t* dst = static_cast<uint8_t*>(o.vhatT) + orow * BKB + part * TOK;
-        const float iv = vinv[c];
-#pragma unroll
-        for (int t0 = 0; t0 < TOK; t0 += 16) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int t = part * TOK + t0 + 4 * u;
-            const uint16_t lo = cvt_e4m3x2(__fmul_rn(vs[t * D + c], iv), __fmul_rn(vs[(t + 1) * D + c], iv));
-            const uint16_t hi = cvt_e4m3x2(__fmul_rn(vs[(t + 2) * D + c], iv), __fmul_rn(vs[(t + 3) * D + c], iv));
-            w[u] = (uint32_t)lo | ((uint32_t)hi << 16);
-          }
-          *reinterpret_cast<uint4*>(dst + t0) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      } else {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.vhatT) + orow * BKB + part * TOK;
-#pragma unroll
-        for (int t0 = 0; t0 < TOK; t0 += 8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int t = part * TOK + t0 + 2 * u;
-            w[u] = cvt_bf16x2(vs[t * D + c], vs[(t + 1) * D + c]);
-          }
-          *reinterpret_cast<uint4*>(dst + t0) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        const float a = __uint_as_float(o.vamax[(size_t)bh * D + eg * 8 + c]);
+        vinv[c] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
       }
     }
-    // z_j
-    if (tid < D) {
-      float z = 0.f;
-      for (int t = 0; t < BKB; ++t) z += phi[t * D + tid];
-      o.z[((size_t)bh * nk + j) * D + tid] = z;
-      zp += z;
+    if (o.quant == 1 && chunk == 0 && tid < D) {
+      const float a = __uint_as_float(o.vamax[(size_t)bh * D + tid]);
+      o.sv[(size_t)bh * D + tid] = a > 0.f ? __fdiv_rn(a, 448.f) : 0.f;
     }
-    // h_j = phi^T V : thread tile rows [ty*T, +T) x cols [tx*T, +T)
-    float acc[T][T];
-#pragma unroll
-    for (int a = 0; a < T; ++a)
-#pragma unroll
-      for (int b = 0; b < T; ++b) acc[a][b] = 0.f;
-    for (int t = 0; t < BKB; ++t) {
-      float pa[T], vb[T];
-#pragma unroll
-      for (int a = 0; a < T; ++a) pa[a] = phi[t * D + ty * T + a];
-#pragma unroll
-      for (int b = 0; b < T; ++b) vb[b] = vs[t * D + tx * T + b];
-#pragma unroll
-      for (int a = 0; a < T; ++a)
-#pragma unroll
-        for (int b = 0; b < T; ++b) acc[a][b] = fmaf(pa[a], vb[b], acc[a][b]);
+    if (D < 128) {   // rows D..127 of the A operand stay zero (the MMA always has M = 128)
+      for (int t = tid; t < (128 - D) * 8; t += 128)
+        *reinterpret_cast<uint4*>(sA + D * 128 + t * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
-    float* hdst = o.h + ((size_t)bh * nk + j) * D * D;
+    float zp = 0.f;                  // this thread's feature (tid < D) partial of Z
+    const uint32_t lane_taddr = tmem + ((uint32_t)(warp * 32) << 16);
+    bool ok = true;
+    for (int n = 0; n < cnt; ++n) {
+      const int j = j0 + n;
+      float* zred = zred_all + (n & 1) * TG * D;
+      float* ared = ared_all + (n & 1) * 4;
+      ok = mbar_wait(tma_full + (n & 1), (n >> 1) & 1, abort_flag, o.status, o.budget_ns);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const uint8_t* sK = base + (n & 1) * C::STAGE;
+      const uint8_t* sV = sK + C::KV_TILE;
+      const size_t rowbase = (size_t)bh * N + (size_t)j * BKB;
+      // ---- K: smooth, K-hat, phi
+      float x[TPT][8];
+      float amax = 0.f;
 #pragma unroll
-    for (int a = 0; a < T; ++a) {
+      for (int u = 0; u < TPT; ++u) {
+        const int t = tg * TPT + u;
+        const uint4 w = *reinterpret_cast<const uint4*>(sK + sl * BKB * 128 + t * 128 + ((ch ^ (t & 7)) << 4));
+        float kv[8];
+        unpack8(w, kv);
 #pragma unroll
-      for (int b = 0; b < T; b += 4) {
-        *reinterpret_cast<float4*>(hdst + (size_t)(ty * T + a) * D + tx * T + b) =
-            make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+        for (int c = 0; c < 8; ++c) {
+          x[u][c] = __fsub_rn(kv[c], cs[c]);
+          amax = fmaxf(amax, fabsf(x[u][c]));
+        }
+      }
+      if (o.khat) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0) ared[warp] = amax;
+        conv_sync();
+        const float a = fmaxf(fmaxf(ared[0], ared[1]), fmaxf(ared[2], ared[3]));
+        const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+#pragma unroll
+        for (int u = 0; u < TPT; ++u) {
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c], inv))));
+            const int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c + 4], inv))));
+            lo |= (uint32_t)(q0 & 0xFF) << (8 * c);
+            hi |= (uint32_t)(q1 & 0xFF) << (8 * c);
+          }
+          *reinterpret_cast<uint2*>(o.khat + (rowbase + tg * TPT + u) * D + eg * 8) = make_uint2(lo, hi);
+        }
+        if (tid == 0) o.sk[(size_t)bh * nk + j] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
+      }
+      float zc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) zc[c] = 0.f;
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) {
+        float m = x[u][0];
+#pragma unroll
+        for (int c = 1; c < 8; ++c) m = fmaxf(m, x[u][c]);
+#pragma unroll
+        for (int off = EG / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          x[u][c] = expf(x[u][c] - m);
+          sum += x[u][c];
+        }
+#pragma unroll
+        for (int off = EG / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float inv = 1.f / sum;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          x[u][c] *= inv;          // phi
+          zc[c] += x[u][c];
+        }
+      }
+      // phi^T operand: row e, tokens tg*TPT .. +TPT (fp16; 128-byte rows, 128-byte swizzle)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int e = eg * 8 + c;
+        const int byte = tg * TPT * 2;
+        uint8_t* dst = sB + e * 128 + ((((byte >> 4) ^ (e & 7))) << 4) + (byte & 15);
+        if constexpr (TPT == 8)
+          *reinterpret_cast<uint4*>(dst) = make_uint4(h2_bits(x[0][c], x[1][c]), h2_bits(x[2][c], x[3][c]),
+                                                      h2_bits(x[4][c], x[5][c]), h2_bits(x[6][c], x[7][c]));
+        else
+          *reinterpret_cast<uint2*>(dst) = make_uint2(h2_bits(x[0][c], x[1][c]), h2_bits(x[2][c], x[3][c]));
+      }
+      // ---- V: V^T operand (fp16), V-hat^T (e4m3) or the bf16 V^T copy
+      float vv[TPT][8];
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) {
+        const int t = tg * TPT + u;
+        const uint4 w = *reinterpret_cast<const uint4*>(sV + sl * BKB * 128 + t * 128 + ((ch ^ (t & 7)) << 4));
+        unpack8(w, vv[u]);
       }
 #pragma unroll
-      for (int b = 0; b < T; ++b) hp[a][b] += acc[a][b];
+      for (int c = 0; c < 8; ++c) {
+        const int cc = eg * 8 + c;
+        const int byte = tg * TPT * 2;
+        uint8_t* dst = sA + cc * 128 + ((((byte >> 4) ^ (cc & 7))) << 4) + (byte & 15);
+        const size_t orow = ((size_t)bh * nk + j) * D + cc;
+        if constexpr (TPT == 8) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(h2_bits(vv[0][c], vv[1][c]), h2_bits(vv[2][c], vv[3][c]),
+                                                      h2_bits(vv[4][c], vv[5][c]), h2_bits(vv[6][c], vv[7][c]));
+        } else {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(h2_bits(vv[0][c], vv[1][c]), h2_bits(vv[2][c], vv[3][c]));
+        }
+        if (o.vhatT) {
+          if (o.quant == 1) {
+            uint32_t wq[TPT / 4];
+#pragma unroll
+            for (int u = 0; u < TPT; u += 4) {
+              const uint16_t p0 = cvt_e4m3x2(__fmul_rn(vv[u][c], vinv[c]), __fmul_rn(vv[u + 1][c], vinv[c]));
+              const uint16_t p1 = cvt_e4m3x2(__fmul_rn(vv[u + 2][c], vinv[c]), __fmul_rn(vv[u + 3][c], vinv[c]));
+              wq[u / 4] = (uint32_t)p0 | ((uint32_t)p1 << 16);
+            }
+            uint8_t* vd = static_cast<uint8_t*>(o.vhatT) + orow * BKB + tg * TPT;
+            if constexpr (TPT == 8)
+              *reinterpret_cast<uint2*>(vd) = make_uint2(wq[0], wq[1]);
+            else
+              *reinterpret_cast<uint32_t*>(vd) = wq[0];
+          } else {
+            __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(o.vhatT) + orow * BKB + tg * TPT;
+            if constexpr (TPT == 8)
+              *reinterpret_cast<uint4*>(vd) = make_uint4(cvt_bf16x2(vv[0][c], vv[1][c]), cvt_bf16x2(vv[2][c], vv[3][c]),
+                                                         cvt_bf16x2(vv[4][c], vv[5][c]), cvt_bf16x2(vv[6][c], vv[7][c]));
+            else
+              *reinterpret_cast<uint2*>(vd) = make_uint2(cvt_bf16x2(vv[0][c], vv[1][c]), cvt_bf16x2(vv[2][c], vv[3][c]));
+          }
+        }
+      }
+      // ---- operands complete: hand them (and the staged tile) to the MMA thread
+#pragma unroll
+      for (int c = 0; c < 8; ++c) zred[tg * D + eg * 8 + c] = zc[c];
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(conv_done);
+      conv_sync();
+      if (tid < D) {
+        float z = 0.f;
+#pragma unroll
+        for (int g = 0; g < TG; ++g) z += zred[g * D + tid];
+        o.z[((size_t)bh * nk + j) * D + tid] = z;
+        zp += z;
+      }
+      // ---- h_j^T: TMEM lane c (one channel per thread) -> global
+      ok = mbar_wait(mma_done, n & 1, abort_flag, o.status, o.budget_ns);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const int c = warp * 32 + lane;
+      if (warp * 32 < D) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(lane_taddr + cc * 32, r);
+          tmem_wait_ld();
+          if (o.h_mode == 1) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+#pragma unroll
+            for (int q = 0; q < 32; q += 8)
+              *reinterpret_cast<uint4*>(dst + q) = make_uint4(
+                  cvt_bf16x2(__uint_as_float(r[q]), __uint_as_float(r[q + 1])),
+                  cvt_bf16x2(__uint_as_float(r[q + 2]), __uint_as_float(r[q + 3])),
+                  cvt_bf16x2(__uint_as_float(r[q + 4]), __uint_as_float(r[q + 5])),
+                  cvt_bf16x2(__uint_as_float(r[q + 6]), __uint_as_float(r[q + 7])));
+          } else {
+            float* dst = static_cast<float*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+#pragma unroll
+            for (int q = 0; q < 32; q += 4)
+              *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                                                __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+          }
+        }
+      }
+      tc_fence_before();
     }
-    __syncthreads();   // before the next block overwrites phi / vs
+    // ---- chunk partials (H^T from the accumulating TMEM columns, Z)
+    if (ok && warp * 32 < D) {
+      const int c = warp * 32 + lane;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(lane_taddr + C::COL_TOT + cc * 32, r);
+        tmem_wait_ld();
+        float* dst = o.hpart + (((size_t)bh * G + chunk) * D + c) * D + cc * 32;
+#pragma unroll
+        for (int q = 0; q < 32; q += 4)
+          *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                                            __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+      }
+    }
+    if (tid < D) o.zpart[((size_t)bh * G + chunk) * D + tid] = zp;
   }
-  float* pdst = o.hpart + ((size_t)bh * G + chunk) * D * D;
-#pragma unroll
-  for (int a = 0; a < T; ++a)
-#pragma unroll
-    for (int b = 0; b < T; b += 4)
-      *reinterpret_cast<float4*>(pdst + (size_t)(ty * T + a) * D + tx * T + b) =
-          make_float4(hp[a][b], hp[a][b + 1], hp[a][b + 2], hp[a][b + 3]);
-  if (tid < D) o.zpart[((size_t)bh * G + chunk) * D + tid] = zp;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
 }
 
 __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const float* __restrict__ zpart, int G, int D,
@@ -226,22 +380,32 @@ __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const floa
   }
 }
 
+constexpr int kSMs = 148;   // B200 streaming multiprocessors
+
 }  // namespace
 
-int linear_chunks(int nk) { return nk < LIN_CHUNKS ? nk : LIN_CHUNKS; }
+int linear_chunks(int BH, int nk) {
+  int G = (2 * kSMs) / BH;   // one wave at two CTAs per SM
+  if (G < 1) G = 1;
+  if (G > nk) G = nk;
+  return G;
+}
 
 cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, const float* c32, const LinearOut& o,
                                 cudaStream_t st) {
-  dim3 grid(linear_chunks(s.nk), s.BH);
-  const size_t smem = (size_t)(2 * BKB * s.d + 2 * s.d + 8) * sizeof(float);
-  auto kb = static_cast<const __nv_bfloat16*>(k);
-  auto vb = static_cast<const __nv_bfloat16*>(v);
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)s.BH * s.N;
+  if (!make_tmap_2d(&tk, k, 2, s.d, rows, 64, BKB, 128) || !make_tmap_2d(&tv, v, 2, s.d, rows, 64, BKB, 128))
+    return cudaErrorInvalidValue;
+  dim3 grid(linear_chunks(s.BH, s.nk), s.BH);
   if (s.d == 128) {
-    cudaFuncSetAttribute(linear_state_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    linear_state_kernel<128><<<grid, LIN_THREADS, smem, st>>>(kb, vb, c32, s.N, s.nk, o);
+    auto kern = linear_state_kernel<128>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LinCfg<128>::SMEM);
+    kern<<<grid, LIN_THREADS, LinCfg<128>::SMEM, st>>>(tk, tv, c32, s.N, s.nk, o);
   } else {
-    cudaFuncSetAttribute(linear_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    linear_state_kernel<64><<<grid, LIN_THREADS, smem, st>>>(kb, vb, c32, s.N, s.nk, o);
+    auto kern = linear_state_kernel<64>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LinCfg<64>::SMEM);
+    kern<<<grid, LIN_THREADS, LinCfg<64>::SMEM, st>>>(tk, tv, c32, s.N, s.nk, o);
   }
   return cudaGetLastError();
 }
@@ -250,7 +414,7 @@ cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float
                                  cudaStream_t st) {
   const int DD = s.d * s.d;
   dim3 grid((DD + 255) / 256, s.BH);
-  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.nk), s.d, Htot, Ztot);
+  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, Htot, Ztot);
   return cudaGetLastError();
 }
 

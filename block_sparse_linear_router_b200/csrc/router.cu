@@ -47,7 +47,7 @@ __device__ __forceinline__ int quant_i8(float x, float inv) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(256, 2) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k,
                                                    const __nv_bfloat16* __restrict__ v, int N, int nq, int nk,
                                                    float* __restrict__ qbar, double* __restrict__ ksum,
@@ -62,15 +62,11 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int cg = tid % TPR, rg = tid / TPR;
   const size_t base = ((size_t)bh * N + (size_t)i * BQ) * D + cg * 8;
 
-  uint4 wq[NP], wk[NP], wv[NP];
+  uint4 wq[NP], wk[NP];
 #pragma unroll
   for (int p = 0; p < NP; ++p) wq[p] = __ldg(reinterpret_cast<const uint4*>(q + base + (size_t)(p * RPP + rg) * D));
 #pragma unroll
   for (int p = 0; p < NP; ++p) wk[p] = __ldg(reinterpret_cast<const uint4*>(k + base + (size_t)(p * RPP + rg) * D));
-  if (vamax) {
-#pragma unroll
-    for (int p = 0; p < NP; ++p) wv[p] = __ldg(reinterpret_cast<const uint4*>(v + base + (size_t)(p * RPP + rg) * D));
-  }
 
   // ---- Q: pooled mean (exact fp64 sum, one rounding to fp32) and INT8 Q-hat
   double cs[8];
@@ -138,6 +134,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 
   // ---- V: per-channel |V| maximum (non-negative floats order like their bits)
   if (vamax) {
+    uint4 wv[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) wv[p] = __ldg(reinterpret_cast<const uint4*>(v + base + (size_t)(p * RPP + rg) * D));
     float vm[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) vm[c] = 0.f;
@@ -161,64 +160,108 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
-__global__ void colmean_kernel(const double* __restrict__ ksum, int nk, int N, int D, double* __restrict__ c64,
-                               float* __restrict__ c32) {
-  const int bh = blockIdx.x;
-  for (int e = threadIdx.x; e < D; e += blockDim.x) {
-    double s = 0.0;
-    for (int j = 0; j < nk; ++j) s += ksum[((size_t)bh * nk + j) * D + e];
-    const double m = s / (double)N;
-    c64[(size_t)bh * D + e] = m;
-    c32[(size_t)bh * D + e] = (float)m;
-  }
-}
-
-constexpr int PROJ_ROWS = 32;
-
-template <int D>
-__global__ void __launch_bounds__(256) proj_kernel(const float* __restrict__ qbar, const double* __restrict__ ksum,
-                                                   const double* __restrict__ c64, const float* __restrict__ wq,
-                                                   const float* __restrict__ wk, int H, int nq, int nk,
-                                                   float* __restrict__ A, float* __restrict__ Bk) {
-  extern __shared__ float psm[];
-  float* W = psm;              // [D][D]
-  float* X = psm + D * D;      // [PROJ_ROWS][D]
-  const int bh = blockIdx.y, h = bh % H, tid = threadIdx.x;
-  const int nqb = (nq + PROJ_ROWS - 1) / PROJ_ROWS;
-  const bool isq = (int)blockIdx.x < nqb;
-  const int r0 = (isq ? blockIdx.x : blockIdx.x - nqb) * PROJ_ROWS;
-  const int nrows = isq ? nq : nk;
-  const float* Wsrc = (isq ? wq : wk) + (size_t)h * D * D;
-  for (int t = tid; t < D * D / 4; t += 256)
-    reinterpret_cast<float4*>(W)[t] = __ldg(reinterpret_cast<const float4*>(Wsrc) + t);
-  for (int t = tid; t < PROJ_ROWS * D; t += 256) {
-    const int r = t / D, e = t % D, row = r0 + r;
-    float x = 0.f;
-    if (row < nrows) {
-      if (isq) {
-        x = qbar[((size_t)bh * nq + row) * D + e];
-      } else {
-        x = (float)(ksum[((size_t)bh * nk + row) * D + e] / (double)BKB - c64[(size_t)bh * D + e]);
-      }
-    }
-    X[t] = x;
+// c = (sum of the exact per-block column sums) / N in fp64, then the smoothed
+// pooled keys Kbar_j - c (fp32). One CTA per (head, 32 columns); 8 warps split
+// the key blocks, partial sums are combined in a fixed order.
+__global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restrict__ ksum, int nk, int N, int D,
+                                                           double* __restrict__ c64, float* __restrict__ c32,
+                                                           float* __restrict__ kbar_s) {
+  __shared__ double part[8][32];
+  __shared__ double cm[32];
+  const int bh = blockIdx.x, col = blockIdx.y * 32 + (threadIdx.x & 31), w = threadIdx.x >> 5;
+  double acc = 0.0;
+  for (int j = w; j < nk; j += 8) acc += ksum[((size_t)bh * nk + j) * D + col];
+  part[w][threadIdx.x & 31] = acc;
+  __syncthreads();
+  if (w == 0) {
+    double t = 0.0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t += part[u][threadIdx.x];
+    const double m = t / (double)N;
+    cm[threadIdx.x] = m;
+    c64[(size_t)bh * D + col] = m;
+    c32[(size_t)bh * D + col] = (float)m;
   }
   __syncthreads();
-  constexpr int GROUPS = 256 / D;
-  constexpr int RPG = PROJ_ROWS / GROUPS;
-  const int col = tid % D, g = tid / D;
-  float* out = isq ? A : Bk;
-  for (int rr = 0; rr < RPG; ++rr) {
-    const int r = g * RPG + rr, row = r0 + r;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int f = 0; f < D; ++f) acc = fmaf(X[r * D + f], W[f * D + col], acc);
-    if (row < nrows) out[((size_t)bh * nrows + row) * D + col] = acc;
+  const double m = cm[threadIdx.x & 31];
+  for (int j = w; j < nk; j += 8) {
+    const size_t o = ((size_t)bh * nk + j) * D + col;
+    kbar_s[o] = (float)(ksum[o] / (double)BKB - m);
   }
 }
 
-constexpr int TOPK_ROWS = 8;          // one warp per query-block row
-constexpr int TOPK_MAX_NK = 6144;     // scores of 8 rows stay in shared memory
+// Batched fp32 SIMT GEMM for the router's small products:
+//   C[b][m][n] = (sum_k X[b][m][k] * Y'[k][n]) / div
+// with Y' = Y[yb]^T (Y stored [N][K], "nt") or Y[yb] (stored [K][N], "nn"),
+// yb = b % ymod. K is the head dimension (a multiple of 32); each product is
+// accumulated sequentially over k in fp32. 64 x 64 tile per CTA, 4 x 4 per thread.
+template <bool NT>
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ X, const float* __restrict__ Y,
+                                                       float* __restrict__ C, int M, int N, int K, int ymod,
+                                                       float div) {
+  __shared__ __align__(16) float Xs[32][68];
+  __shared__ __align__(16) float Ys[32][68];
+  const int b = blockIdx.z, yb = b % ymod, tid = threadIdx.x;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int ty = tid >> 4, tx = tid & 15;
+  const float* Xb = X + (size_t)b * M * K;
+  const float* Yb = Y + (size_t)yb * N * K;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    // X tile: 64 rows x 32 k -> Xs[k][m]
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int t = tid + u * 256, r = t >> 3, kq = (t & 7) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m0 + r < M) v = *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + r) * K + k0 + kq);
+      Xs[kq][r] = v.x; Xs[kq + 1][r] = v.y; Xs[kq + 2][r] = v.z; Xs[kq + 3][r] = v.w;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int t = tid + u * 256;
+      if (NT) {
+        const int r = t >> 3, kq = (t & 7) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + r < N) v = *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq);
+        Ys[kq][r] = v.x; Ys[kq + 1][r] = v.y; Ys[kq + 2][r] = v.z; Ys[kq + 3][r] = v.w;
+      } else {
+        const int kk = t >> 4, nq4 = (t & 15) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (n0 + nq4 < N) v = *reinterpret_cast<const float4*>(Yb + (size_t)(k0 + kk) * N + n0 + nq4);
+        *reinterpret_cast<float4*>(&Ys[kk][nq4]) = v;
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&Xs[kk][ty * 4]);
+      const float4 bb = *reinterpret_cast<const float4*>(&Ys[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) C[((size_t)b * M + m) * N + n] = div == 1.f ? acc[i][j] : __fdiv_rn(acc[i][j], div);
+    }
+  }
+}
+
+constexpr int TOPK_WARPS = 4;         // one warp per query-block row
+constexpr int TOPK_MAX_NK = 6144;     // a row's order keys stay in shared memory
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -226,73 +269,48 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) scores_topk_kernel(const float* __restrict__ A, const float* __restrict__ Bk,
-                                                          int nq, int nk, int k, uint8_t* __restrict__ mask,
-                                                          int32_t* __restrict__ idx, float* __restrict__ scores) {
-  extern __shared__ float tsm[];
-  float* As = tsm;                          // [TOPK_ROWS][D]
-  float* Bt = As + TOPK_ROWS * D;           // [D][33]
-  float* sc = Bt + D * 33;                  // [TOPK_ROWS][nk]
-  const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row0 = blockIdx.x * TOPK_ROWS, row = row0 + warp;
-  const bool valid = row < nq;
-  for (int t = tid; t < TOPK_ROWS * D; t += 256) {
-    const int r = t / D;
-    As[t] = (row0 + r < nq) ? A[((size_t)bh * nq + row0) * D + t] : 0.f;
-  }
-  const float sqrt_d = sqrtf((float)D);
-  for (int jt = 0; jt < nk; jt += 32) {
-    __syncthreads();
-    for (int t = tid; t < 32 * D; t += 256) {
-      const int jj = t / D, e = t % D;
-      Bt[e * 33 + jj] = (jt + jj < nk) ? Bk[((size_t)bh * nk + jt + jj) * D + e] : 0.f;
-    }
-    __syncthreads();
-    if (valid && jt + lane < nk) {
-      float acc = 0.f;
-#pragma unroll 8
-      for (int e = 0; e < D; ++e) acc = fmaf(As[warp * D + e], Bt[e * 33 + lane], acc);
-      sc[warp * nk + jt + lane] = __fdiv_rn(acc, sqrt_d);
-    }
-  }
+// Hard top-k of one logit row per warp: the k-th largest order key by a
+// bitwise search from the top bit down, then an ascending ballot compaction
+// that keeps every key above it and the lowest-indexed keys equal to it.
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ scores, int rows, int nk,
+                                                               int k, uint8_t* __restrict__ mask,
+                                                               int32_t* __restrict__ idx) {
+  extern __shared__ uint32_t keys_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * TOPK_WARPS + warp;
+  if (row >= rows) return;
+  uint32_t* keys = keys_all + (size_t)warp * nk;
+  const float* s = scores + (size_t)row * nk;
+  for (int j = lane; j < nk; j += 32) keys[j] = order_key(s[j]);
   __syncwarp();
-  if (!valid) return;
-  const float* s = sc + warp * nk;
-  // k-th largest key by a bitwise search from the top bit down
   uint32_t T = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
     int cnt = 0;
-    for (int j = lane; j < nk; j += 32) cnt += order_key(s[j]) >= cand;
+    for (int j = lane; j < nk; j += 32) cnt += keys[j] >= cand;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     if (cnt >= k) T = cand;
   }
   int gt = 0;
-  for (int j = lane; j < nk; j += 32) gt += order_key(s[j]) > T;
+  for (int j = lane; j < nk; j += 32) gt += keys[j] > T;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
-  const int need = k - gt;          // how many entries equal to T are kept (lowest indices first)
+  const int need = k - gt;          // entries equal to T that are kept (lowest indices first)
   const uint32_t lt = (1u << lane) - 1u;
   int eq_seen = 0, pos = 0;
-  const size_t rbase = (size_t)bh * nq + row;
   for (int jb = 0; jb < nk; jb += 32) {
     const int j = jb + lane;
     const bool in = j < nk;
-    const float sv = in ? s[j] : 0.f;
-    const uint32_t key = in ? order_key(sv) : 0u;
+    const uint32_t key = in ? keys[j] : 0u;
     const bool is_gt = in && key > T;
     const bool is_eq = in && key == T;
     const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
     const bool sel = is_gt || (is_eq && (eq_seen + __popc(eqm & lt)) < need);
     eq_seen += __popc(eqm);
     const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-    if (in) {
-      mask[rbase * nk + j] = sel ? 1 : 0;
-      if (scores) scores[rbase * nk + j] = sv;
-    }
-    if (sel) idx[rbase * k + pos + __popc(selm & lt)] = j;
+    if (in) mask[(size_t)row * nk + j] = sel ? 1 : 0;
+    if (sel) idx[(size_t)row * k + pos + __popc(selm & lt)] = j;
     pos += __popc(selm);
   }
 }
@@ -312,39 +330,41 @@ cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void
   return cudaGetLastError();
 }
 
-cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, cudaStream_t st) {
-  colmean_kernel<<<s.BH, 128, 0, st>>>(ksum, s.nk, s.N, s.d, c64, c32);
+cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, float* kbar_s,
+                           cudaStream_t st) {
+  colmean_kbar_kernel<<<dim3(s.BH, s.d / 32), 256, 0, st>>>(ksum, s.nk, s.N, s.d, c64, c32, kbar_s);
   return cudaGetLastError();
 }
 
-cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const double* ksum, const double* c64,
-                          const float* wq, const float* wk, float* A, float* Bk, cudaStream_t st) {
-  const int nb = (s.nq + PROJ_ROWS - 1) / PROJ_ROWS + (s.nk + PROJ_ROWS - 1) / PROJ_ROWS;
-  dim3 grid(nb, s.BH);
-  const size_t smem = (size_t)(s.d * s.d + PROJ_ROWS * s.d) * sizeof(float);
-  if (s.d == 128) {
-    cudaFuncSetAttribute(proj_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    proj_kernel<128><<<grid, 256, smem, st>>>(qbar, ksum, c64, wq, wk, H, s.nq, s.nk, A, Bk);
-  } else {
-    cudaFuncSetAttribute(proj_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    proj_kernel<64><<<grid, 256, smem, st>>>(qbar, ksum, c64, wq, wk, H, s.nq, s.nk, A, Bk);
-  }
+static cudaError_t gemm(bool nt, const float* X, const float* Y, float* C, int batch, int M, int N, int K, int ymod,
+                        float div, cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64, batch);
+  if (nt)
+    gemm_f32_kernel<true><<<grid, 256, 0, st>>>(X, Y, C, M, N, K, ymod, div);
+  else
+    gemm_f32_kernel<false><<<grid, 256, 0, st>>>(X, Y, C, M, N, K, ymod, div);
   return cudaGetLastError();
+}
+
+cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const float* kbar_s, const float* wq,
+                        const float* wk, float* A, float* Bk, cudaStream_t st) {
+  cudaError_t e = gemm(false, qbar, wq, A, s.BH, s.nq, s.d, s.d, H, 1.f, st);
+  if (e != cudaSuccess) return e;
+  return gemm(false, kbar_s, wk, Bk, s.BH, s.nk, s.d, s.d, H, 1.f, st);
+}
+
+cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float* scores, cudaStream_t st) {
+  return gemm(true, A, Bk, scores, s.BH, s.nq, s.nk, s.d, s.BH, sqrtf((float)s.d), st);
 }
 
 int scores_topk_max_nk() { return TOPK_MAX_NK; }
 
-cudaError_t launch_scores_topk(const Shape& s, const float* A, const float* Bk, uint8_t* mask, int32_t* idx,
-                               float* scores_opt, cudaStream_t st) {
-  dim3 grid((s.nq + TOPK_ROWS - 1) / TOPK_ROWS, s.BH);
-  const size_t smem = (size_t)(TOPK_ROWS * s.d + s.d * 33 + TOPK_ROWS * s.nk) * sizeof(float);
-  if (s.d == 128) {
-    cudaFuncSetAttribute(scores_topk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    scores_topk_kernel<128><<<grid, 256, smem, st>>>(A, Bk, s.nq, s.nk, s.k, mask, idx, scores_opt);
-  } else {
-    cudaFuncSetAttribute(scores_topk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    scores_topk_kernel<64><<<grid, 256, smem, st>>>(A, Bk, s.nq, s.nk, s.k, mask, idx, scores_opt);
-  }
+cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st) {
+  const int rows = s.BH * s.nq;
+  const size_t smem = (size_t)TOPK_WARPS * s.nk * sizeof(uint32_t);
+  cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  topk_kernel<<<(rows + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(scores, rows, s.nk, s.k, mask,
+                                                                                   idx);
   return cudaGetLastError();
 }
 

@@ -148,7 +148,8 @@ def router(q, k, proj_q, proj_k, frac, workspace: Optional[Workspace] = None, sc
 
 
 def linear_state(k, v, colmean, workspace: Optional[Workspace] = None, stream=None):
-    """h_j, z_j, H_total, Z_total (fp32) for smoothed keys K - colmean."""
+    """Per key block h_j^T (fp32 [B,H,nk,d(c),d(e)]), z_j, and their sums H_total^T, Z_total, for the
+    smoothed keys K - colmean."""
     lib = load_library()
     _check_qkv(k, v, colmean)
     B, H, N, d = k.shape

@@ -114,11 +114,15 @@ sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k,
 /* Step 3's per-key-block linear-attention state (detail page §7, note 2:
  * h_j precomputed per key block, then accumulated):
  *   phi(x) = softmax over the d features; K_s = K - colmean (fp32)
- *   h_out    : fp32 [B][H][N/64][d][d], h_j = phi(K_s,j)^T V_j
+ *   h_out    : fp32 [B][H][N/64][d][d], TRANSPOSED: h_out[..][j][c][e] =
+ *              sum over the block's tokens t of V[t][c] * phi(K_s[t])[e]
+ *              (= (phi(K_s,j)^T V_j)^T; tensor-core products with fp16
+ *              operands, fp32 accumulation)
  *   z_out    : fp32 [B][H][N/64][d],    z_j = column sums of phi(K_s,j)
- *   Htot_out : fp32 [B][H][d][d] = sum_j h_j;  Ztot_out: fp32 [B][H][d]
+ *   Htot_out : fp32 [B][H][d][d] = sum_j h_out[j] (same transposed layout)
+ *   Ztot_out : fp32 [B][H][d] = sum_j z_j
  *   colmean  : fp32 [B][H][d] as returned by sla2_router.
- * Uses desc->workspace for the partial sums. */
+ * Uses desc->workspace for the per-chunk partial sums. */
 sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v,
                               const float* colmean, float* h_out, float* z_out,
                               float* Htot_out, float* Ztot_out, void* stream);

@@ -104,7 +104,7 @@ def _compare_full(sla2, inp, frac, tag):
     if errs["ol"]:
         e_ol = rel_l2(np.concatenate([a for a, _ in errs["ol"]]), np.concatenate([b for _, b in errs["ol"]]))
         print(f"[{tag}] rel-L2 O_l={e_ol:.2e}")
-        assert e_ol <= 1e-4
+        assert e_ol <= 1e-3    # tf32 phi(Q) H_i product, bf16 h_j storage
     return e_o
 
 
@@ -175,8 +175,9 @@ def test_router_entry_point(sla2):
     np.testing.assert_array_equal(r["colmean"].cpu().numpy(), cm.astype(np.float32))
 
 
-def test_linear_state_entry_point(sla2):
-    inp = make_custom(1, 2, 1024, 64, 0.1, seed=29)
+@pytest.mark.parametrize("d", [64, 128])
+def test_linear_state_entry_point(sla2, d):
+    inp = make_custom(1, 2, 1024, d, 0.1, seed=29)
     dev = to_dev(inp)
     cm = sla2.router(dev["q"], dev["k"], dev["proj_q"], dev["proj_k"], 0.1)["colmean"]
     st = sla2.linear_state(dev["k"], dev["v"], cm)
@@ -184,9 +185,12 @@ def test_linear_state_entry_point(sla2):
         K = inp.k[0, h].double().numpy()
         V = inp.v[0, h].double().numpy()
         hh, zz = O.linear_states(K - O.colmean(K), V)
-        assert rel_l2(st["h"][0, h].cpu().numpy(), hh) < 1e-5
+        hT = hh.transpose(0, 2, 1)                       # the library stores h_j^T
+        e_h = rel_l2(st["h"][0, h].cpu().numpy(), hT)
+        print(f"linear state d={d} head {h}: rel-L2 h {e_h:.2e}")
+        assert e_h < 1e-3                                # fp16 phi operand, fp32 accumulation
         assert rel_l2(st["z"][0, h].cpu().numpy(), zz) < 1e-5
-        assert rel_l2(st["Htot"][0, h].cpu().numpy(), hh.sum(0)) < 1e-5
+        assert rel_l2(st["Htot"][0, h].cpu().numpy(), hT.sum(0)) < 1e-3
         assert rel_l2(st["Ztot"][0, h].cpu().numpy(), zz.sum(0)) < 1e-5
 
 
