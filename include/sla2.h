@@ -111,6 +111,33 @@ sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k,
                         uint8_t* mask_out, int32_t* idx_out, float* colmean_out,
                         void* stream);
 
+/* The router of sla2_router, for callers that cannot allocate device memory
+ * (no counterpart on the SLA2 pages; an addition of this library). Some
+ * callers may not call cudaMalloc at all: a plugin inside a host framework
+ * that owns every device allocation (for instance a serving runtime with a
+ * pre-sized memory pool), or code on a latency-critical path where an
+ * allocation, which can synchronise the device, is not allowed. This entry
+ * point allocates nothing: its scratch is a fixed device array of
+ * SLA2_ROUTER_NOALLOC_SCRATCH_BYTES compiled into libsla2.so, which every GPU
+ * that loads the library holds until the process exits.
+ *   - Arguments and outputs are those of sla2_router; desc->workspace is
+ *     ignored (desc->dbg_scores is honoured).
+ *   - Shapes whose router scratch exceeds the array are rejected with
+ *     SLA2_ERR_WORKSPACE before anything is launched. The scratch is about
+ *     (5/16) N d + N^2 / 2048 bytes per (batch, head): 1.84 MB for N = 32768,
+ *     d = 128, so up to 8 such heads fit in one call.
+ *   - The first call on each device looks up the array's device address with
+ *     cudaGetSymbolAddress while that device is current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it has to start at zero). Calls whose kernels may overlap on
+ *     the GPU (other streams, other host threads) race on it: serialise them. */
+#define SLA2_ROUTER_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+sla2_status sla2_router_noalloc(const sla2_desc* desc, const void* q, const void* k,
+                                const float* proj_q, const float* proj_k, float topk_frac,
+                                uint8_t* mask_out, int32_t* idx_out, float* colmean_out,
+                                void* stream);
+
 /* Step 3's per-key-block linear-attention state (detail page §7, note 2:
  * h_j precomputed per key block, then accumulated):
  *   phi(x) = softmax over the d features; K_s = K - colmean (fp32)
