@@ -54,7 +54,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 // Workspace regions (each 256-byte aligned).
 struct Layout {
   size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
-      os, total;
+      zscale, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -90,6 +90,7 @@ Layout make_layout(const Shape& s, int quant) {
   L.zpart = take(BH * G * d * 4);
   L.Htot = take(BH * d * d * 4);
   L.Ztot = take(BH * d * 4);
+  L.zscale = take(BH * 4);
   L.os = take(BH * N * d * 4);
   L.total = off;
   return L;
@@ -236,7 +237,7 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
   o.status = desc->status;
   o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
-  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, Htot_out, Ztot_out, st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, Htot_out, Ztot_out, at<float>(desc, L.zscale), st));
   return SLA2_OK;
 }
 
@@ -285,7 +286,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   o.status = desc->status;
   o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
-  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, at<float>(desc, L.Htot), at<float>(desc, L.Ztot), st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
+                                at<float>(desc, L.zscale), st));
   SLA2_TRY(mark(2));
 
   // sparse branch: tensor maps over the (quantised) operands
@@ -314,6 +316,7 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.q = q;
   ea.Htot = at<float>(desc, L.Htot);
   ea.Ztot = at<float>(desc, L.Ztot);
+  ea.zscale = at<float>(desc, L.zscale);
   ea.hT = at<uint16_t>(desc, L.h);
   ea.z = o.z;
   ea.idx = idx;
@@ -325,7 +328,10 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  SLA2_TRY(launch_epilogue(s, ea, st));
+  CUtensorMap tqe;
+  if (!make_map(&tqe, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B))
+    return SLA2_ERR_CUDA;
+  SLA2_TRY(launch_epilogue(s, ea, tqe, st));
   SLA2_TRY(mark(4));
 
   // debug exports

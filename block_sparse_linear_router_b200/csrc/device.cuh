@@ -92,6 +92,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// 1-D bulk copy global -> shared of `bytes` (multiple of 16; both addresses
+// 16-byte aligned), completion counted in bytes on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -164,19 +172,29 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t dfmt, uint32_t afmt, uint32_t bfmt, uint32_t M, uint32_t N) {
   return (dfmt << 4) | (afmt << 7) | (bfmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
+// The same with both operands MN-major (bit 15: A, bit 16: B).
+__host__ __device__ constexpr uint32_t make_idesc_mn(uint32_t dfmt, uint32_t afmt, uint32_t bfmt, uint32_t M,
+                                                     uint32_t N) {
+  return make_idesc(dfmt, afmt, bfmt, M, N) | (1u << 15) | (1u << 16);
+}
 
 // Shared-memory matrix descriptor for a K-major, swizzled operand tile:
-//   bits 0-13 start address >> 4; 16-29 leading byte offset >> 4 (unused by
-//   swizzled K-major layouts, set to 1); 32-45 stride byte offset >> 4 (distance
-//   between consecutive 8-row groups); 46-47 version = 1; 61-63 layout
-//   (2 = 128-byte swizzle, 4 = 64-byte swizzle). Tiles are 1024-byte aligned, so
-//   the base-offset field stays 0. Moving along K inside a swizzle atom is done
-//   by advancing the start address.
+//   bits 0-13 start address >> 4; 16-29 leading byte offset >> 4; 32-45 stride
+//   byte offset >> 4; 46-47 version = 1; 61-63 layout (2 = 128-byte swizzle,
+//   4 = 64-byte swizzle). Tiles are 1024-byte aligned, so the base-offset field
+//   stays 0.
+//   K-major swizzled operand: rows of 128 (or 64) bytes along K; SBO = distance
+//   between consecutive 8-row groups; LBO unused (16). Moving along K inside a
+//   swizzle atom is done by advancing the start address.
+//   MN-major swizzled operand: 128-byte rows along M/N, one row per K index;
+//   SBO = distance between consecutive groups of 8 K rows, LBO = distance
+//   between consecutive 128-byte column blocks along M/N.
 enum : uint32_t { LAYOUT_SW128 = 2u, LAYOUT_SW64 = 4u };
-__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_bytes, uint32_t layout) {
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_bytes, uint32_t layout,
+                                               uint32_t lbo_bytes = 16) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(layout & 7u) << 61;

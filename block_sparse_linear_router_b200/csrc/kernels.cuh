@@ -61,7 +61,7 @@ int linear_chunks(int BH, int nk);
 cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, const float* c32, const LinearOut& o,
                                 cudaStream_t st);
 cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, float* Htot, float* Ztot,
-                                 cudaStream_t st);
+                                 float* zscale, cudaStream_t st);
 
 // ---- sparse branch (sparse.cu) --------------------------------------------
 struct SparseArgs {
@@ -83,6 +83,7 @@ struct EpilogueArgs {
   const void* q;        // bf16 [BH][N][d]
   const float* Htot;    // H_total^T [BH][d][d] (fp32)
   const float* Ztot;    // [BH][d]
+  const float* zscale;  // [BH] power of two with Z_total * zscale <= 1
   const uint16_t* hT;   // h_j^T bf16 [BH][nk][d][d]
   const float* z;       // [BH][nk][d]
   const int32_t* idx;   // [BH][nq][k]
@@ -95,6 +96,6 @@ struct EpilogueArgs {
   unsigned* status;
   unsigned long long budget_ns;
 };
-cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st);
+cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, const CUtensorMap& tq, cudaStream_t st);
 
 }  // namespace sla2

@@ -13,9 +13,13 @@
 //   h_j^T = V_j^T phi_j  on the tensor core: tcgen05 kind::f16 with fp16
 //           operands (V exactly, phi rounded once), fp32 accumulation in TMEM;
 //           a second TMEM accumulator sums h_j^T over the chunk (partial H^T).
-// Roles: warps 0-3 convert (TMA-staged bf16 tiles -> operands, quantised
-// copies, phi, z) and read results back from TMEM; warp 4 lane 0 issues the
-// TMA loads (two stages) and the MMAs.
+// The staged tiles are [token][column] with 128-byte swizzle, which is the
+// MN-major operand layout: the converters overwrite K with phi (fp16) and V
+// with V (fp16) in place, and the MMA reads them as A = V (M = channel) and
+// B = phi (N = feature), both MN-major, K = the 64 tokens.
+// Roles: warps 0-3 convert (quantised copies, phi, z, fp16 operands) and read
+// results back from TMEM; warp 4 lane 0 issues the TMA loads (two stages) and
+// the MMAs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -30,18 +34,18 @@ constexpr int LIN_THREADS = 160;     // 4 converter warps + 1 TMA / MMA warp
 
 template <int D>
 struct LinCfg {
-  static constexpr int SLABS = D / 64;                 // 64 bf16 = 128-byte slabs of a staged K/V tile
-  static constexpr int KV_TILE = BKB * D * 2;          // bytes of one staged bf16 K (or V) tile
-  static constexpr int STAGE = 2 * KV_TILE;            // K + V
+  static constexpr int SLABS = D / 64;                 // 64-column (128-byte) slabs of a staged tile
+  static constexpr int SLAB = BKB * 128;               // one slab: 64 tokens x 128 bytes
+  static constexpr int KV_TILE = SLABS * SLAB;         // bytes of one staged bf16 K (or V) tile
+  static constexpr int OFF_V = KV_TILE;                // V tile (then a zero slab when D = 64: M is 128)
+  static constexpr int STAGE = KV_TILE + 2 * SLAB;
   static constexpr int EG = D / 8;                     // feature groups of 8 per token row
   static constexpr int TG = 128 / EG;                  // token groups
   static constexpr int TPT = BKB / TG;                 // tokens per converter thread
-  static constexpr int OFF_A = 2 * STAGE;              // V^T operand (MMA A: M = 128 rows, channels c < D)
-  static constexpr int OFF_B = OFF_A + 128 * 128;      // phi^T operand (MMA B: N = D rows of features e)
-  static constexpr int OFF_RED = OFF_B + D * 128;      // z partials [2][TG][D] + amax [2][4]
+  static constexpr int OFF_RED = 2 * STAGE;            // z partials [2][TG][D] + amax [2][4]
   static constexpr int OFF_BAR = OFF_RED + (2 * TG * D + 8) * 4;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;
-  static constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
+  static constexpr uint32_t IDESC = make_idesc_mn(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
   static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
   static constexpr uint32_t COL_TOT = D;                // running partial H^T
 };
@@ -69,8 +73,6 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   using C = LinCfg<D>;
   extern __shared__ uint8_t lsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = base + C::OFF_A;
-  uint8_t* sB = base + C::OFF_B;
   float* zred_all = reinterpret_cast<float*>(base + C::OFF_RED);     // [2][TG][D]
   float* ared_all = zred_all + 2 * C::TG * D;                        // [2][4]
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
@@ -109,30 +111,34 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       auto load = [&](int n) {
         uint8_t* stg = base + (n & 1) * C::STAGE;
         const int row = bh * N + (j0 + n) * BKB;
-        mbar_arrive_expect_tx(tma_full + (n & 1), C::STAGE);
+        mbar_arrive_expect_tx(tma_full + (n & 1), 2 * C::KV_TILE);
 #pragma unroll
         for (int sl = 0; sl < C::SLABS; ++sl) {
-          tma_load_2d(stg + sl * BKB * 128, &tk, tma_full + (n & 1), sl * 64, row);
-          tma_load_2d(stg + C::KV_TILE + sl * BKB * 128, &tv, tma_full + (n & 1), sl * 64, row);
+          tma_load_2d(stg + sl * C::SLAB, &tk, tma_full + (n & 1), sl * 64, row);
+          tma_load_2d(stg + C::OFF_V + sl * C::SLAB, &tv, tma_full + (n & 1), sl * 64, row);
         }
       };
       load(0);
       if (cnt > 1) load(1);
-      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+      bool ok = true;
       for (int n = 0; n < cnt; ++n) {
-        if (!mbar_wait(conv_done, n & 1, abort_flag, o.status, o.budget_ns)) break;
-        if (n + 2 < cnt) load(n + 2);      // stage n & 1 has been read
+        if (!mbar_wait(conv_done, n & 1, abort_flag, o.status, o.budget_ns)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t stg = smem_u32(base + (n & 1) * C::STAGE);
 #pragma unroll
-        for (int ks = 0; ks < BKB / 16; ++ks) {
-          const uint64_t ad = make_sdesc(a0 + ks * 32, 1024, LAYOUT_SW128);
-          const uint64_t bd = make_sdesc(b0 + ks * 32, 1024, LAYOUT_SW128);
+        for (int ks = 0; ks < BKB / 16; ++ks) {      // 16 tokens = two 8-row groups per MMA
+          const uint64_t ad = make_sdesc(stg + C::OFF_V + ks * 2048, 1024, LAYOUT_SW128, C::SLAB);
+          const uint64_t bd = make_sdesc(stg + ks * 2048, 1024, LAYOUT_SW128, C::SLAB);
           mma_f16(tmem, ad, bd, C::IDESC, ks > 0);
           mma_f16(tmem + C::COL_TOT, ad, bd, C::IDESC, (n > 0 || ks > 0));
         }
         tc_commit(mma_done);
+        if (n + 2 < cnt) {                           // the stage is free once the MMA has read it
+          if (!mbar_wait(mma_done, n & 1, abort_flag, o.status, o.budget_ns)) { ok = false; break; }
+          load(n + 2);
+        }
       }
-      if (*(volatile int*)abort_flag) {
+      if (!ok) {
         // let in-flight copies land and issued MMAs finish before the CTA releases its memory
         for (int n = (cnt > 2 ? cnt - 2 : 0); n < cnt; ++n) mbar_wait_drain(tma_full + (n & 1), (n >> 1) & 1, 20000000ull);
         tc_commit(bar + 6);
@@ -160,9 +166,10 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       const float a = __uint_as_float(o.vamax[(size_t)bh * D + tid]);
       o.sv[(size_t)bh * D + tid] = a > 0.f ? __fdiv_rn(a, 448.f) : 0.f;
     }
-    if (D < 128) {   // rows D..127 of the A operand stay zero (the MMA always has M = 128)
-      for (int t = tid; t < (128 - D) * 8; t += 128)
-        *reinterpret_cast<uint4*>(sA + D * 128 + t * 16) = make_uint4(0u, 0u, 0u, 0u);
+    if (D < 128) {   // channels D..127 of the A operand are a zero slab (the MMA always has M = 128)
+      for (int st = 0; st < 2; ++st)
+        for (int t = tid; t < C::SLAB / 16; t += 128)
+          *reinterpret_cast<uint4*>(base + st * C::STAGE + C::OFF_V + C::KV_TILE + t * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
     float zp = 0.f;                  // this thread's feature (tid < D) partial of Z
     const uint32_t lane_taddr = tmem + ((uint32_t)(warp * 32) << 16);
@@ -173,8 +180,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       float* ared = ared_all + (n & 1) * 4;
       ok = mbar_wait(tma_full + (n & 1), (n >> 1) & 1, abort_flag, o.status, o.budget_ns);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      const uint8_t* sK = base + (n & 1) * C::STAGE;
-      const uint8_t* sV = sK + C::KV_TILE;
+      uint8_t* sK = base + (n & 1) * C::STAGE;
+      uint8_t* sV = sK + C::OFF_V;
       const size_t rowbase = (size_t)bh * N + (size_t)j * BKB;
       // ---- K: smooth, K-hat, phi
       float x[TPT][8];
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
 #pragma unroll
       for (int u = 0; u < TPT; ++u) {
         const int t = tg * TPT + u;
-        const uint4 w = *reinterpret_cast<const uint4*>(sK + sl * BKB * 128 + t * 128 + ((ch ^ (t & 7)) << 4));
+        const uint4 w = *reinterpret_cast<const uint4*>(sK + sl * C::SLAB + t * 128 + ((ch ^ (t & 7)) << 4));
         float kv[8];
         unpack8(w, kv);
 #pragma unroll
@@ -237,39 +244,28 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
           zc[c] += x[u][c];
         }
       }
-      // phi^T operand: row e, tokens tg*TPT .. +TPT (fp16; 128-byte rows, 128-byte swizzle)
+      // phi (fp16) in place over the staged K tile: the MMA's B operand
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int e = eg * 8 + c;
-        const int byte = tg * TPT * 2;
-        uint8_t* dst = sB + e * 128 + ((((byte >> 4) ^ (e & 7))) << 4) + (byte & 15);
-        if constexpr (TPT == 8)
-          *reinterpret_cast<uint4*>(dst) = make_uint4(h2_bits(x[0][c], x[1][c]), h2_bits(x[2][c], x[3][c]),
-                                                      h2_bits(x[4][c], x[5][c]), h2_bits(x[6][c], x[7][c]));
-        else
-          *reinterpret_cast<uint2*>(dst) = make_uint2(h2_bits(x[0][c], x[1][c]), h2_bits(x[2][c], x[3][c]));
+      for (int u = 0; u < TPT; ++u) {
+        const int t = tg * TPT + u;
+        *reinterpret_cast<uint4*>(sK + sl * C::SLAB + t * 128 + ((ch ^ (t & 7)) << 4)) =
+            make_uint4(h2_bits(x[u][0], x[u][1]), h2_bits(x[u][2], x[u][3]), h2_bits(x[u][4], x[u][5]),
+                       h2_bits(x[u][6], x[u][7]));
       }
-      // ---- V: V^T operand (fp16), V-hat^T (e4m3) or the bf16 V^T copy
+      // ---- V: fp16 in place (the MMA's A operand), V-hat^T (e4m3) or the bf16 V^T copy
       float vv[TPT][8];
 #pragma unroll
       for (int u = 0; u < TPT; ++u) {
         const int t = tg * TPT + u;
-        const uint4 w = *reinterpret_cast<const uint4*>(sV + sl * BKB * 128 + t * 128 + ((ch ^ (t & 7)) << 4));
-        unpack8(w, vv[u]);
+        uint4* p = reinterpret_cast<uint4*>(sV + sl * C::SLAB + t * 128 + ((ch ^ (t & 7)) << 4));
+        unpack8(*p, vv[u]);
+        *p = make_uint4(h2_bits(vv[u][0], vv[u][1]), h2_bits(vv[u][2], vv[u][3]), h2_bits(vv[u][4], vv[u][5]),
+                        h2_bits(vv[u][6], vv[u][7]));
       }
+      if (o.vhatT) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int cc = eg * 8 + c;
-        const int byte = tg * TPT * 2;
-        uint8_t* dst = sA + cc * 128 + ((((byte >> 4) ^ (cc & 7))) << 4) + (byte & 15);
-        const size_t orow = ((size_t)bh * nk + j) * D + cc;
-        if constexpr (TPT == 8) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(h2_bits(vv[0][c], vv[1][c]), h2_bits(vv[2][c], vv[3][c]),
-                                                      h2_bits(vv[4][c], vv[5][c]), h2_bits(vv[6][c], vv[7][c]));
-        } else {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(h2_bits(vv[0][c], vv[1][c]), h2_bits(vv[2][c], vv[3][c]));
-        }
-        if (o.vhatT) {
+        for (int c = 0; c < 8; ++c) {
+          const size_t orow = ((size_t)bh * nk + j) * D + eg * 8 + c;
           if (o.quant == 1) {
             uint32_t wq[TPT / 4];
 #pragma unroll
@@ -363,8 +359,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   }
 }
 
+// H_total^T and Z_total as fixed-order sums of the chunk partials, plus a
+// per-head power of two 2^-E >= ... with max_e Z_total[e] <= 2^E, which the
+// epilogue applies to H_i and Z_i so that both fit fp16 operands exactly
+// scaled (the ratio H_i / Z_i does not change).
 __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const float* __restrict__ zpart, int G, int D,
-                                     float* __restrict__ Htot, float* __restrict__ Ztot) {
+                                     float* __restrict__ Htot, float* __restrict__ Ztot, float* __restrict__ zscale) {
+  __shared__ float zmax[8];
   const int bh = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int DD = D * D;
@@ -373,10 +374,24 @@ __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const floa
     for (int g = 0; g < G; ++g) s += hpart[((size_t)bh * G + g) * DD + e];
     Htot[(size_t)bh * DD + e] = s;
   }
-  if (blockIdx.x == 0 && threadIdx.x < D) {
+  if (blockIdx.x == 0) {
     float s = 0.f;
-    for (int g = 0; g < G; ++g) s += zpart[((size_t)bh * G + g) * D + threadIdx.x];
-    Ztot[(size_t)bh * D + threadIdx.x] = s;
+    if (threadIdx.x < D) {
+      for (int g = 0; g < G; ++g) s += zpart[((size_t)bh * G + g) * D + threadIdx.x];
+      Ztot[(size_t)bh * D + threadIdx.x] = s;
+    }
+    float m = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) zmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0 && zscale) {
+      float mx = 0.f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, zmax[w]);
+      int ex = 0;
+      frexpf(mx, &ex);                       // mx = f * 2^ex, f in [0.5, 1)
+      zscale[bh] = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
+    }
   }
 }
 
@@ -411,10 +426,10 @@ cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, co
 }
 
 cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, float* Htot, float* Ztot,
-                                 cudaStream_t st) {
+                                 float* zscale, cudaStream_t st) {
   const int DD = s.d * s.d;
   dim3 grid((DD + 255) / 256, s.BH);
-  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, Htot, Ztot);
+  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, Htot, Ztot, zscale);
   return cudaGetLastError();
 }
 

@@ -221,3 +221,42 @@ def test_bounded_wait_reports_timeout_and_context_survives(sla2):
     sla2.forward(dev["q"], dev["k"], dev["v"], dev["proj_q"], dev["proj_k"], dev["alpha"], 0.25, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 3, 8192, 128, 0.03), (1, 3, 8192, 64, 0.1)])
+def test_more_query_blocks_than_sms(sla2, shape):
+    """192 (head, query block) items: the persistent epilogue walks several
+    items per CTA and the linear-state pass splits heads into chunks."""
+    B, H, N, d, frac = shape
+    _compare_full(sla2, make_custom(B, H, N, d, frac, seed=32), frac, f"multiwave-d{d}")
+
+
+def test_full_size_wan13b_sampled(sla2):
+    """The benchmarked workload (Wan2.1-1.3B shape: 1 x 12 x 32768 x 128, k% = 3)
+    in the same launch configuration as bench.py: the whole mask against the
+    oracle router, and the output on sampled query blocks of sampled heads."""
+    w = WORKLOADS["wan1.3b"]
+    inp = make_inputs(w)
+    dev = to_dev(inp)
+    out, dbg = sla2.forward(dev["q"], dev["k"], dev["v"], dev["proj_q"], dev["proj_k"], dev["alpha"],
+                            w.topk_frac, quantize=1, out_dtype=torch.bfloat16, debug=True)
+    torch.cuda.synchronize()
+    k = O.topk_count(w.nk, w.topk_frac)
+    mask, idx, scores = O.router(inp.q, inp.k, inp.proj_q, inp.proj_k, w.topk_frac)
+    near = check_mask_rows(dbg["mask"].cpu().numpy(), mask, scores, k)
+    go = out.float().cpu().numpy()
+    rng = np.random.default_rng(0)
+    errs = []
+    for h in (0, 5, 11):
+        blocks = sorted(rng.choice(w.nq, size=4, replace=False).tolist())
+        blocks = [i for i in blocks if (0, h, i) not in near]
+        r = O.head_forward(*head_np(inp, 0, h), w.topk_frac, mode="qa", blocks=blocks)
+        for n, i in enumerate(blocks):
+            got = go[0, h, i * 128:(i + 1) * 128]
+            ref = r["O"][n * 128:(n + 1) * 128]
+            errs.append((got, ref))
+    g = np.concatenate([a for a, _ in errs])
+    rf = np.concatenate([b for _, b in errs])
+    e, m = rel_l2(g, rf), float(np.max(np.abs(g - rf)))
+    print(f"[wan1.3b sampled] rel-L2 {e:.2e} max-abs {m:.2e} near-tie rows {len(near)}")
+    assert e <= REL_L2_Q and m <= MAX_ABS_Q
