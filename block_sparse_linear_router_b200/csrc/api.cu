@@ -8,7 +8,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/sla2.h"
+#include "sla2.h"
 #include "device.cuh"
 #include "kernels.cuh"
 

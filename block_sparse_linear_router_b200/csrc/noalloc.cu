@@ -20,7 +20,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/sla2.h"
+#include "sla2.h"
 #include "kernels.cuh"
 
 namespace {

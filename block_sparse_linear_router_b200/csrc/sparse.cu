@@ -3,18 +3,26 @@
 // over the selected entries, O_s = dequant(P-hat V-hat); SLA2 detail page §7
 // note 2: only the selected block pairs are computed).
 //
-// One CTA per (head, query block), heads outermost so a head's key blocks stay
-// in L2 while its query blocks run. 192 threads in four roles:
+// Persistent CTAs (two per SM) walk the (head, query block) items in
+// head-major order, so the SMs work on neighbouring query blocks of the same
+// head and the head's K/V blocks stay in L2. Each item is one 128-row query
+// block and its k selected 64-token key blocks, visited in ascending order.
+// Tensor memory and barriers are set up once; barrier phases run on across
+// items (g counts key blocks over all items of the CTA). 192 threads:
 //   warps 0-3  softmax: thread t owns query row t (= TMEM lane t); online
-//              softmax with one running-max update per key block, P written
-//              to shared memory as e4m3 (x448 fixed scale) or bf16, O rescaled
-//              in TMEM when a row max grows, final normalisation and store.
-//   warp 4     TMA producer: Q tile once, then (K_j, V_j^T) per selected j
-//              into a ring of NS stages (no multicast).
-//   warp 5     tcgen05 issuer: S_n = Q K_j^T into one of two TMEM buffers
-//              (kind::i8 -> s32, or kind::f16 -> f32), then O += P_n V_j
-//              (kind::f8f6f4 e4m3 or kind::f16 bf16 -> f32 TMEM); QK for the
-//              next block is issued before PV of the current one.
+//              softmax with one running-max update per key block; P written
+//              to shared memory as e4m3 (x448 fixed scale) or bf16; O rescaled
+//              in TMEM when a row max grows; at the end of an item the row is
+//              normalised and stored while the next item's S is computed.
+//   warp 4     TMA producer: per item the Q tile (double-buffered, prefetched
+//              one item ahead); K_j and V_j^T of each selected j into separate
+//              rings of NS stages (no multicast): a K stage is released when
+//              its QK has finished, a V stage when its PV has, and V is loaded
+//              one block behind K because PV runs two blocks behind QK.
+//   warp 5     tcgen05 issuer, in the order QK(g), PV(g-2): S_g = Q K_j^T into
+//              one of two TMEM buffers (kind::i8 -> s32, or kind::f16 -> f32)
+//              as soon as that buffer's previous S has been read, and
+//              O += P_g V_j (kind::f8f6f4 e4m3 or kind::f16 bf16 -> f32).
 // TMEM columns: [0,64) S buffer 0, [64,128) S buffer 1, [128,128+D) O.
 #include <cuda_bf16.h>
 
@@ -28,7 +36,10 @@ namespace {
 template <int D, bool QUANT>
 struct Cfg {
   static constexpr int ESZ = QUANT ? 1 : 2;                 // bytes per element of Q/K/V/P
-  static constexpr int NS = QUANT ? 3 : 2;                  // K/V ring depth
+  static constexpr int NS = 3;                              // depth of the K ring and of the V ring
+  // V(g) is loaded after K(g+1) and needs PV(g - NS) done, which the issuer
+  // starts before QK(g+1): NS >= 3 keeps the issue orders free of a cycle
+  static_assert(NS >= 3, "ring depth");
   static constexpr int QK_ROW = D * ESZ;                    // bytes of one Q/K row
   static constexpr int QK_SW = QK_ROW >= 128 ? 128 : 64;    // swizzle span of Q/K tiles
   static constexpr int QK_PARTS = QK_ROW / QK_SW;           // 128-byte column slabs of a Q/K tile
@@ -41,14 +52,15 @@ struct Cfg {
   static constexpr int PV_STEPS = VP_ROW / 32;
   static constexpr uint32_t QK_LAYOUT = QK_SW == 128 ? LAYOUT_SW128 : LAYOUT_SW64;
   static constexpr uint32_t VP_LAYOUT = VP_ROW == 128 ? LAYOUT_SW128 : LAYOUT_SW64;
-  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int OFF_K = 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * K_BYTES;
   static constexpr int OFF_P = OFF_V + NS * V_BYTES;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_empty[2], p_full[2], pv_done
-  static constexpr int NBAR = 1 + 2 * NS + 6 + 1;
-  static constexpr int OFF_SV = OFF_BAR + 8 * 16;
-  static constexpr int OFF_MISC = OFF_SV + 4 * D;
+  // barriers: q_full[2], q_free[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
+  //           s_full[2], s_empty[2], p_full[2], p_free[2], o_full, o_free, drain
+  static constexpr int NBAR = 4 + 4 * NS + 8 + 3;
+  static_assert(NBAR <= 32, "barrier region");
+  static constexpr int OFF_MISC = OFF_BAR + ((8 * NBAR + 15) / 16) * 16;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + alignment slack
   static constexpr uint32_t IDESC_QK = QUANT ? make_idesc(2, 1, 1, 128, 64) : make_idesc(1, 1, 1, 128, 64);
   static constexpr uint32_t IDESC_PV = QUANT ? make_idesc(1, 0, 0, 128, D) : make_idesc(1, 1, 1, 128, D);
@@ -68,47 +80,57 @@ constexpr uint64_t DRAIN_NS = 20000000ull;   // 20 ms for in-flight copies / MMA
 
 template <int D, bool QUANT>
 __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid_constant__ CUtensorMap tq,
-                                                        const __grid_constant__ CUtensorMap tk,
-                                                        const __grid_constant__ CUtensorMap tv, Shape s,
-                                                        SparseArgs a) {
+                                                                    const __grid_constant__ CUtensorMap tk,
+                                                                    const __grid_constant__ CUtensorMap tv, Shape s,
+                                                                    SparseArgs a) {
   using C = Cfg<D, QUANT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = base;
   uint8_t* sK = base + C::OFF_K;
   uint8_t* sV = base + C::OFF_V;
   uint8_t* sP = base + C::OFF_P;
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
-  uint64_t* q_full = bar;
-  uint64_t* kv_full = bar + 1;
-  uint64_t* kv_empty = bar + 1 + C::NS;
-  uint64_t* s_full = bar + 1 + 2 * C::NS;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* pv_done = s_full + 6;
-  uint64_t* drain = s_full + 7;
-  float* s_sv = reinterpret_cast<float*>(base + C::OFF_SV);
+  uint64_t* q_full = bar;                     // [2]
+  uint64_t* q_free = bar + 2;                 // [2]
+  uint64_t* k_full = bar + 4;                 // [NS]
+  uint64_t* k_empty = k_full + C::NS;         // [NS]
+  uint64_t* v_full = k_empty + C::NS;         // [NS]
+  uint64_t* v_empty = v_full + C::NS;         // [NS]
+  uint64_t* s_full = v_empty + C::NS;         // [2]
+  uint64_t* s_empty = s_full + 2;             // [2]
+  uint64_t* p_full = s_full + 4;              // [2]
+  uint64_t* p_free = s_full + 6;              // [2]: the PV reading P buffer b has finished
+  uint64_t* o_full = s_full + 8;              // the last PV of an item has finished
+  uint64_t* o_free = s_full + 9;              // the softmax warps have read O of the item
+  uint64_t* drain = s_full + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(base + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / s.nq, qi = blockIdx.x % s.nq;
   const int k = s.k;
-  const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * k;
+  const int total = s.BH * s.nq;
+  const int nitems = total > (int)blockIdx.x ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int nblocks = nitems * k;             // key blocks over all of this CTA's items
   volatile int* abortf = abort_flag;
+  auto item_of = [&](int it) { return (int)blockIdx.x + it * (int)gridDim.x; };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int st = 0; st < C::NS; ++st) {
-      mbar_init(kv_full + st, 1);
-      mbar_init(kv_empty + st, 1);
-    }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full + b, 1);
+      mbar_init(q_free + b, 1);
       mbar_init(s_full + b, 1);
-      mbar_init(s_empty + b, 128);
-      mbar_init(p_full + b, 128);
+      mbar_init(s_empty + b, 4);     // one arrival per softmax warp
+      mbar_init(p_full + b, 4);
+      mbar_init(p_free + b, 1);
     }
-    mbar_init(pv_done, 1);
+    for (int st = 0; st < C::NS; ++st) {
+      mbar_init(k_full + st, 1);
+      mbar_init(k_empty + st, 1);
+      mbar_init(v_full + st, 1);
+      mbar_init(v_empty + st, 1);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -117,9 +139,6 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (QUANT && threadIdx.x < 128) {
-    for (int e = threadIdx.x; e < D; e += 128) s_sv[e] = a.sv[(size_t)bh * D + e];
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -127,49 +146,94 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
 
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && nitems > 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      const int qrow = bh * s.N + qi * BQ;
-      mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-#pragma unroll
-      for (int part = 0; part < C::QK_PARTS; ++part)
-        tma_load_2d(sQ + part * BQ * C::QK_SW, &tq, q_full, part * (C::QK_SW / C::ESZ), qrow);
-      int issued = 0;
-      for (int n = 0; n < k; ++n) {
-        const int st = n % C::NS;
-        if (n >= C::NS && !mbar_wait(kv_empty + st, ((n / C::NS) - 1) & 1, abortf, a.status, a.budget_ns)) break;
-        ++issued;
-        const int j = __ldg(sel + n);
-        mbar_arrive_expect_tx(kv_full + st, C::K_BYTES + C::V_BYTES);
+      int g = 0, qissued = 0;
+      bool ok = true;
+      auto load_q = [&](int it) -> bool {
+        const int b = it & 1;
+        if (it >= 2 && !mbar_wait(q_free + b, ((it >> 1) - 1) & 1, abortf, a.status, a.budget_ns)) return false;
+        const int w = item_of(it);
+        const int bh = w / s.nq, qi = w % s.nq;
+        mbar_arrive_expect_tx(q_full + b, C::Q_BYTES);
 #pragma unroll
         for (int part = 0; part < C::QK_PARTS; ++part)
-          tma_load_2d(sK + st * C::K_BYTES + part * BKB * C::QK_SW, &tk, kv_full + st, part * (C::QK_SW / C::ESZ),
-                      bh * s.N + j * BKB);
-        tma_load_2d(sV + st * C::V_BYTES, &tv, kv_full + st, 0, (bh * s.nk + j) * D);
+          tma_load_2d(base + b * C::Q_BYTES + part * BQ * C::QK_SW, &tq, q_full + b, part * (C::QK_SW / C::ESZ),
+                      bh * s.N + qi * BQ);
+        ++qissued;
+        return true;
+      };
+      ok = load_q(0);
+      int gv = 0;                            // V blocks issued (V trails K by one block)
+      int bh_prev = 0, j_prev = 0;
+      auto load_v = [&](int bh, int j) -> bool {
+        const int st = gv % C::NS;
+        if (gv >= C::NS && !mbar_wait(v_empty + st, ((gv / C::NS) - 1) & 1, abortf, a.status, a.budget_ns)) return false;
+        mbar_arrive_expect_tx(v_full + st, C::V_BYTES);
+        tma_load_2d(sV + st * C::V_BYTES, &tv, v_full + st, 0, (bh * s.nk + j) * D);
+        ++gv;
+        return true;
+      };
+      for (int it = 0; ok && it < nitems; ++it) {
+        const int w = item_of(it);
+        const int bh = w / s.nq, qi = w % s.nq;
+        const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * k;
+        int j_next = __ldg(sel);
+        for (int n = 0; n < k; ++n) {
+          const int st = g % C::NS;
+          const int j = j_next;
+          if (n + 1 < k) j_next = __ldg(sel + n + 1);
+          if (g >= C::NS && !mbar_wait(k_empty + st, ((g / C::NS) - 1) & 1, abortf, a.status, a.budget_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(k_full + st, C::K_BYTES);
+#pragma unroll
+          for (int part = 0; part < C::QK_PARTS; ++part)
+            tma_load_2d(sK + st * C::K_BYTES + part * BKB * C::QK_SW, &tk, k_full + st,
+                        part * (C::QK_SW / C::ESZ), bh * s.N + j * BKB);
+          ++g;
+          if (g >= 2 && !load_v(bh_prev, j_prev)) {
+            ok = false;
+            break;
+          }
+          bh_prev = bh;
+          j_prev = j;
+          // prefetch the next item's Q once this item's first K block is on its way
+          if (n == 0 && it + 1 < nitems && !load_q(it + 1)) {
+            ok = false;
+            break;
+          }
+        }
       }
-      if (*abortf) {
-        // let the copies still in flight land before the CTA's shared memory is released
-        mbar_wait_drain(q_full, 0, DRAIN_NS);
-        for (int n = issued > C::NS ? issued - C::NS : 0; n < issued; ++n)
-          mbar_wait_drain(kv_full + n % C::NS, (n / C::NS) & 1, DRAIN_NS);
+      if (ok && g > 0) ok = load_v(bh_prev, j_prev);
+      if (!ok) {   // let the copies still in flight land before shared memory is released
+        for (int q = (g > C::NS ? g - C::NS : 0); q < g; ++q)
+          mbar_wait_drain(k_full + q % C::NS, (q / C::NS) & 1, DRAIN_NS);
+        for (int q = (gv > C::NS ? gv - C::NS : 0); q < gv; ++q)
+          mbar_wait_drain(v_full + q % C::NS, (q / C::NS) & 1, DRAIN_NS);
+        for (int q = (qissued > 2 ? qissued - 2 : 0); q < qissued; ++q)
+          mbar_wait_drain(q_full + (q & 1), (q >> 1) & 1, DRAIN_NS);
       }
     }
     __syncwarp();
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV), p_addr = smem_u32(sP);
-      auto issue_qk = [&](int n) -> bool {
-        const int st = n % C::NS, b = n & 1;
-        if (!mbar_wait(kv_full + st, (n / C::NS) & 1, abortf, a.status, a.budget_ns)) return false;
-        if (n >= 2 && !mbar_wait(s_empty + b, ((n - 2) >> 1) & 1, abortf, a.status, a.budget_ns)) return false;
+    if (lane == 0 && nitems > 0) {
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), p_addr = smem_u32(sP);
+      auto issue_qk = [&](int g) -> bool {
+        const int it = g / k, n = g - it * k;
+        const int st = g % C::NS, b = g & 1, qb = it & 1;
+        if (n == 0 && !mbar_wait(q_full + qb, (it >> 1) & 1, abortf, a.status, a.budget_ns)) return false;
+        if (!mbar_wait(k_full + st, (g / C::NS) & 1, abortf, a.status, a.budget_ns)) return false;
+        if (g >= 2 && !mbar_wait(s_empty + b, ((g >> 1) - 1) & 1, abortf, a.status, a.budget_ns)) return false;
         tc_fence_after();
-        const uint32_t kt = k_addr + st * C::K_BYTES;
+        const uint32_t qt = smem_u32(base + qb * C::Q_BYTES), kt = k_addr + st * C::K_BYTES;
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
-          const uint64_t ad = make_sdesc(kstep_addr<C::QK_SW>(q_addr, BQ, ks), 8 * C::QK_SW, C::QK_LAYOUT);
+          const uint64_t ad = make_sdesc(kstep_addr<C::QK_SW>(qt, BQ, ks), 8 * C::QK_SW, C::QK_LAYOUT);
           const uint64_t bd = make_sdesc(kstep_addr<C::QK_SW>(kt, BKB, ks), 8 * C::QK_SW, C::QK_LAYOUT);
           if (QUANT)
             mma_i8(tmem + b * 64, ad, bd, C::IDESC_QK, ks > 0);
@@ -177,11 +241,17 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
             mma_f16(tmem + b * 64, ad, bd, C::IDESC_QK, ks > 0);
         }
         tc_commit(s_full + b);
+        tc_commit(k_empty + st);
+        if (n == k - 1) tc_commit(q_free + qb);      // the item's Q tile has been read
         return true;
       };
-      auto issue_pv = [&](int n) -> bool {
-        const int st = n % C::NS, b = n & 1;
-        if (!mbar_wait(p_full + b, (n >> 1) & 1, abortf, a.status, a.budget_ns)) return false;
+      auto issue_pv = [&](int g) -> bool {
+        const int it = g / k, n = g - it * k;
+        const int st = g % C::NS, b = g & 1;
+        if (!mbar_wait(v_full + st, (g / C::NS) & 1, abortf, a.status, a.budget_ns)) return false;
+        if (!mbar_wait(p_full + b, (g >> 1) & 1, abortf, a.status, a.budget_ns)) return false;
+        // the first PV of an item overwrites O: the previous item's O must have been read
+        if (n == 0 && it > 0 && !mbar_wait(o_free, (it - 1) & 1, abortf, a.status, a.budget_ns)) return false;
         tc_fence_after();
         const uint32_t pt = p_addr + b * C::P_BYTES, vt = v_addr + st * C::V_BYTES;
 #pragma unroll
@@ -193,20 +263,16 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
           else
             mma_f16(tmem + C::COL_O, ad, bd, C::IDESC_PV, (n > 0 || ks > 0));
         }
-        tc_commit(kv_empty + st);
-        tc_commit(pv_done);
+        tc_commit(v_empty + st);
+        tc_commit(p_free + b);
+        if (n == k - 1) tc_commit(o_full);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, abortf, a.status, a.budget_ns);
-      if (ok) {
-        tc_fence_after();
-        ok = issue_qk(0);
+      bool ok = true;
+      for (int g = 0; ok && g < nblocks + 2; ++g) {
+        if (g < nblocks) ok = issue_qk(g);
+        if (ok && g >= 2) ok = issue_pv(g - 2);
       }
-      for (int n = 1; ok && n < k; ++n) {
-        ok = issue_qk(n);
-        if (ok) ok = issue_pv(n - 1);
-      }
-      if (ok) ok = issue_pv(k - 1);
       if (!ok) {
         // wait for every MMA issued so far before the tensor memory is released
         tc_commit(drain);
@@ -220,100 +286,174 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     constexpr float LOG2E = 1.4426950408889634f;
     const float rs_d = rsqrtf((float)D);
-    const float sq_i = QUANT ? a.sq[(size_t)bh * s.nq + qi] : 1.f;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int n = 0; n < k; ++n) {
-      const int b = n & 1;
-      ok = mbar_wait(s_full + b, (n >> 1) & 1, abortf, a.status, a.budget_ns);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_empty + b);
-
-      float scale;   // logits in log2 units = raw * scale
-      if (QUANT) {
-        const int j = __ldg(sel + n);
-        scale = sq_i * __ldg(a.sk + (size_t)bh * s.nk + j) * rs_d * LOG2E;
-      } else {
-        scale = rs_d * LOG2E;
-      }
-      float x[64];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = QUANT ? (float)(int)sr[c] : __uint_as_float(sr[c]);
-        x[c] *= scale;
-        mx = fmaxf(mx, x[c]);
-      }
-      const float m_new = fmaxf(m, mx);
-      const float corr = ex2_approx(m - m_new);     // 0 on the first block
-      float rowsum = 0.f;
-      uint32_t pk[QUANT ? 16 : 32];
-#pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const float p0 = ex2_approx(x[c] - m_new), p1 = ex2_approx(x[c + 1] - m_new);
-        const float p2 = ex2_approx(x[c + 2] - m_new), p3 = ex2_approx(x[c + 3] - m_new);
-        rowsum += (p0 + p1) + (p2 + p3);
-        if (QUANT) {
-          const uint16_t lo = cvt_e4m3x2(448.f * p0, 448.f * p1);
-          const uint16_t hi = cvt_e4m3x2(448.f * p2, 448.f * p3);
-          pk[c / 4] = (uint32_t)lo | ((uint32_t)hi << 16);
-        } else {
-          pk[c / 2] = cvt_bf16x2(p0, p1);
-          pk[c / 2 + 1] = cvt_bf16x2(p2, p3);
-        }
-      }
-      l = l * corr + rowsum;
-      m = m_new;
-      // P buffer b was last read by PV n-2; O must be final for PV n-1 before rescaling
-      if (n >= 1) {
-        ok = mbar_wait(pv_done, (n - 1) & 1, abortf, a.status, a.budget_ns);
+    int g = 0;
+    for (int it = 0; ok && it < nitems; ++it) {
+      const int w = item_of(it);
+      const int bh = w / s.nq, qi = w % s.nq;
+      const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * k;
+      const float sq_i = QUANT ? __ldg(a.sq + (size_t)bh * s.nq + qi) : 1.f;
+      float m = -INFINITY, l = 0.f;
+      // K-block scales prefetched two blocks ahead (their loads depend on the index list)
+      const float* skh = a.sk + (size_t)bh * s.nk;
+      float sk_cur = QUANT ? __ldg(skh + __ldg(sel)) : 1.f;
+      float sk_nxt = (QUANT && k > 1) ? __ldg(skh + __ldg(sel + 1)) : 1.f;
+      for (int n = 0; n < k; ++n, ++g) {
+        const int b = g & 1;
+        const int j2 = (QUANT && n + 2 < k) ? __ldg(sel + n + 2) : 0;
+        ok = mbar_wait(s_full + b, (g >> 1) & 1, abortf, a.status, a.budget_ns);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-      }
-      uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
-      if (QUANT) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int pc = ch ^ ((r >> 1) & 3);        // 64-byte swizzle
-          *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        uint32_t sr[64];
+        tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty + b);
+
+        // logits in log2 units = raw * scale
+        const float scale = QUANT ? sq_i * sk_cur * rs_d * LOG2E : rs_d * LOG2E;
+        if (QUANT) {
+          sk_cur = sk_nxt;
+          sk_nxt = n + 2 < k ? __ldg(skh + j2) : 1.f;
         }
-      } else {
+        // Raw logits as fp32 pairs. For INT8 the s32 accumulator plus 0x4B400000 is
+        // the bit pattern of 12582912 + S exactly (|S| < 2^22); subtracting
+        // 12582912 is exact too, so S becomes a float without an int->float
+        // conversion.
+        uint64_t f2[32];
+        const uint64_t off2 = f2_pack(-12582912.f, -12582912.f);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int pc = ch ^ (r & 7);               // 128-byte swizzle
-          *reinterpret_cast<uint4*>(prow + pc * 16) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int c = 0; c < 32; ++c) {
+          if (QUANT)
+            f2[c] = f2_add(f2_pack(__uint_as_float(sr[2 * c] + 0x4B400000u), __uint_as_float(sr[2 * c + 1] + 0x4B400000u)),
+                           off2);
+          else
+            f2[c] = f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
         }
-      }
-      if (n >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+        float mx8[8];
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + C::COL_O + cc * 32, o);
+        for (int c = 0; c < 8; ++c) {
+          float x0, x1, y0, y1;
+          f2_unpack(f2[c], x0, x1);
+          f2_unpack(f2[c + 8], y0, y1);
+          mx8[c] = fmax3(x0, x1, fmaxf(y0, y1));
+        }
+#pragma unroll
+        for (int c = 16; c < 32; c += 2) {
+          float x0, x1, y0, y1;
+          f2_unpack(f2[c], x0, x1);
+          f2_unpack(f2[c + 1], y0, y1);
+          const int q = (c - 16) >> 1;
+          mx8[q] = fmax3(mx8[q], x0, fmax3(x1, y0, y1));
+        }
+        const float mxf = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_new = fmaxf(m, mxf * scale);
+        const float corr = ex2_approx(m - m_new);     // 0 on the first block
+        // exponent of p = fma(S, scale, c2); the quantised path yields 448 p directly
+        const float c2 = QUANT ? 8.807354922057604f - m_new : -m_new;
+        const uint64_t sc2 = f2_pack(scale, scale), cc2 = f2_pack(c2, c2);
+        uint64_t rs2a = f2_pack(0.f, 0.f), rs2b = f2_pack(0.f, 0.f);
+        uint32_t pk[QUANT ? 16 : 32];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float t0, t1, t2, t3;
+          f2_unpack(f2_fma(f2[c], sc2, cc2), t0, t1);
+          f2_unpack(f2_fma(f2[c + 1], sc2, cc2), t2, t3);
+          const float p0 = ex2_approx(t0), p1 = ex2_approx(t1), p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+          rs2a = f2_add(rs2a, f2_pack(p0, p1));
+          rs2b = f2_add(rs2b, f2_pack(p2, p3));
+          if (QUANT) {
+            const uint16_t lo = cvt_e4m3x2(p0, p1);
+            const uint16_t hi = cvt_e4m3x2(p2, p3);
+            pk[c / 2] = (uint32_t)lo | ((uint32_t)hi << 16);
+          } else {
+            pk[c] = cvt_bf16x2(p0, p1);
+            pk[c + 1] = cvt_bf16x2(p2, p3);
+          }
+        }
+        float ra0, ra1;
+        f2_unpack(f2_add(rs2a, rs2b), ra0, ra1);
+        l = l * corr + (ra0 + ra1);
+        m = m_new;
+        // O must be rescaled by corr (after PV n-1 has finished) before PV n adds to it
+        if (n >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
+          ok = mbar_wait(p_free + ((g - 1) & 1), ((g - 1) >> 1) & 1, abortf, a.status, a.budget_ns);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t o0[32], o1[32], o2[32], o3[32];
+          tmem_ld32(lane_addr + C::COL_O, o0);
+          if (D > 32) tmem_ld32(lane_addr + C::COL_O + 32, o1);
+          if (D > 64) {
+            tmem_ld32(lane_addr + C::COL_O + 64, o2);
+            tmem_ld32(lane_addr + C::COL_O + 96, o3);
+          }
           tmem_wait_ld();
+          const uint64_t corr2 = f2_pack(corr, corr);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-          tmem_st32(lane_addr + C::COL_O + cc * 32, o);
+          for (int c = 0; c < 32; c += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o0[c]), __uint_as_float(o0[c + 1])), corr2), x0, x1);
+            o0[c] = __float_as_uint(x0);
+            o0[c + 1] = __float_as_uint(x1);
+            if (D > 32) {
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o1[c]), __uint_as_float(o1[c + 1])), corr2), x0, x1);
+              o1[c] = __float_as_uint(x0);
+              o1[c + 1] = __float_as_uint(x1);
+            }
+            if (D > 64) {
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o2[c]), __uint_as_float(o2[c + 1])), corr2), x0, x1);
+              o2[c] = __float_as_uint(x0);
+              o2[c + 1] = __float_as_uint(x1);
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o3[c]), __uint_as_float(o3[c + 1])), corr2), x0, x1);
+              o3[c] = __float_as_uint(x0);
+              o3[c + 1] = __float_as_uint(x1);
+            }
+          }
+          tmem_st32(lane_addr + C::COL_O, o0);
+          if (D > 32) tmem_st32(lane_addr + C::COL_O + 32, o1);
+          if (D > 64) {
+            tmem_st32(lane_addr + C::COL_O + 64, o2);
+            tmem_st32(lane_addr + C::COL_O + 96, o3);
+          }
+          tmem_wait_st();
         }
-        tmem_wait_st();
+        // P buffer b was last read by PV g-2
+        if (g >= 2) {
+          ok = mbar_wait(p_free + b, ((g >> 1) - 1) & 1, abortf, a.status, a.budget_ns);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
+        if (QUANT) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int pc = ch ^ ((r >> 1) & 3);        // 64-byte swizzle
+            *reinterpret_cast<uint4*>(prow + pc * 16) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int pc = ch ^ (r & 7);               // 128-byte swizzle
+            *reinterpret_cast<uint4*>(prow + pc * 16) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + b);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full + b);
-    }
-    if (ok) {
-      ok = mbar_wait(pv_done, (k - 1) & 1, abortf, a.status, a.budget_ns);
+      if (!ok) break;
+      // ---- item done: normalise O and store it, then hand O back to the MMA issuer
+      ok = mbar_wait(o_full, it & 1, abortf, a.status, a.budget_ns);
       ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / l;     // quantised path: l holds 448 x the row sum
       float* orow = a.os + ((size_t)bh * s.N + (size_t)qi * BQ + r) * D;
+      const float* svh = a.sv + (size_t)bh * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -323,12 +463,15 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float acc = __uint_as_float(o[c]);
-          v[c] = QUANT ? acc * s_sv[cc * 32 + c] * (1.f / 448.f) * inv_l : acc * inv_l;
+          v[c] = QUANT ? acc * __ldg(svh + cc * 32 + c) * inv_l : acc * inv_l;
         }
 #pragma unroll
         for (int c = 0; c < 32; c += 4)
           *reinterpret_cast<float4*>(orow + cc * 32 + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
     }
   }
 
@@ -340,6 +483,8 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
   }
 }
 
+constexpr int kSMs = 148;   // B200 streaming multiprocessors
+
 template <int D, bool QUANT>
 cudaError_t launch_t(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const SparseArgs& a, cudaStream_t st) {
@@ -347,7 +492,10 @@ cudaError_t launch_t(const Shape& s, const CUtensorMap& tq, const CUtensorMap& t
   auto kern = sparse_kernel<D, QUANT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<s.BH * s.nq, 192, C::SMEM, st>>>(tq, tk, tv, s, a);
+  const int total = s.BH * s.nq;
+  const int per_sm = QUANT ? 2 : 1;
+  const int grid = total < per_sm * kSMs ? total : per_sm * kSMs;
+  kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, s, a);
   return cudaGetLastError();
 }
 

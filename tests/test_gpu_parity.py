@@ -104,7 +104,7 @@ def _compare_full(sla2, inp, frac, tag):
     if errs["ol"]:
         e_ol = rel_l2(np.concatenate([a for a, _ in errs["ol"]]), np.concatenate([b for _, b in errs["ol"]]))
         print(f"[{tag}] rel-L2 O_l={e_ol:.2e}")
-        assert e_ol <= 1e-3    # tf32 phi(Q) H_i product, bf16 h_j storage
+        assert e_ol <= 1e-3    # fp16 phi(Q) H_i product, bf16 h_j storage
     return e_o
 
 
