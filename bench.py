@@ -57,13 +57,20 @@ def work_model(w, k):
         "effective_ops": 4 * B * H * N * N * d,
         # router: read Q, K, V (bf16), write Q-hat (int8)
         "router_bytes": 2 * E * 3 + E,
-        # linear state: read K, V (bf16), write K-hat, V-hat^T (8-bit), h_j^T (bf16), z_j (fp32)
+        # linear state: read K, V (bf16), write K-hat, V-hat^T (8-bit), h_j^T tiles (fp16), z_j (fp32)
         "linear_bytes": 2 * E * 2 + 2 * E + BH * nk * d * d * 2 + BH * nk * d * 4,
-        # epilogue: read Q (bf16), O_s (fp32), h_j^T once (bf16), write out (bf16); the
-        # repeated h_j^T gather (k per query block) is L2 traffic, reported separately
+        # epilogue: read Q (bf16), O_s (fp32), h_j^T tiles once (fp16), write out (bf16); the
+        # repeated tile gather (k + 1 per query block) is L2 traffic, reported separately
         "epilogue_bytes": 2 * E + 4 * E + 2 * E + BH * nk * d * d * 2,
-        "gather_bytes": BH * nq * k * d * d * 2,
+        "gather_bytes": BH * nq * (k + 1) * d * d * 2,   # per query block: H_total and the k selected h_j tiles
     }
+
+
+def launches_per_forward(w, k):
+    """Kernels one forward launches: router 6 (pool, column means, two projections,
+    logits, top-k), linear state 2, sparse 1, Z_i 1 and epilogue 1 (no Z_i pass when
+    every key block is selected)."""
+    return 6 + 2 + 1 + (2 if k < w.N // 64 else 1)
 
 
 class ClockSampler:
@@ -349,7 +356,7 @@ def main():
         "config": {"workload": f"{w.name} B={w.B} H={w.H} N={w.N} d={w.d} k%={w.topk_frac * 100:g} (k={k} of {w.nk})",
                    "l2": "no flush: Q/K/V 302 MB > 126 MB L2", "parallelism": f"replicas x{ws}"},
         "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 8 * K, "clocks": clk,
+        "gpu_launches": launches_per_forward(w, k) * K, "clocks": clk,
         "sparse_issued_tops": kern["sparse"]["achieved"],
     }
     print(json.dumps(line), flush=True)

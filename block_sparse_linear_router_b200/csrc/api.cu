@@ -54,7 +54,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 // Workspace regions (each 256-byte aligned).
 struct Layout {
   size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
-      zscale, os, total;
+      htile, hscale, Zi, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -84,13 +84,15 @@ Layout make_layout(const Shape& s, int quant) {
   L.sk = take(BH * nk * 4);
   L.vhatT = take(BH * nk * d * BKB * (quant ? 1 : 2));
   L.sv = take(BH * d * 4);
-  L.h = take(BH * nk * d * d * 2);   // bf16 h_j^T
+  L.h = take(BH * nk * d * d * 2);   // fp16 -s h_j^T operand tiles
   L.z = take(BH * nk * d * 4);
   L.hpart = take(BH * G * d * d * 4);
   L.zpart = take(BH * G * d * 4);
   L.Htot = take(BH * d * d * 4);
   L.Ztot = take(BH * d * 4);
-  L.zscale = take(BH * 4);
+  L.htile = take(BH * d * d * 2);    // fp16 s H_total^T operand tiles
+  L.hscale = take(BH * 4);
+  L.Zi = take(BH * nq * d * 4);
   L.os = take(BH * N * d * 4);
   L.total = off;
   return L;
@@ -153,10 +155,11 @@ sla2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA2_OK : SLA
 sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
                        const void* v, const float* wq, const float* wk, uint8_t* mask, int32_t* idx, int quant,
                        cudaStream_t st) {
-  if (quant) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
-  SLA2_TRY(launch_pool(s, q, k, quant ? v : nullptr, at<float>(d, L.qbar), at<double>(d, L.ksum),
+  // with V given, its per-channel |V| max (V-hat scales, fp16 scale of the linear state)
+  if (v) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
+  SLA2_TRY(launch_pool(s, q, k, v, at<float>(d, L.qbar), at<double>(d, L.ksum),
                        quant ? at<int8_t>(d, L.qhat) : nullptr, at<float>(d, L.sq),
-                       quant ? at<unsigned>(d, L.vamax) : nullptr, st));
+                       v ? at<unsigned>(d, L.vamax) : nullptr, st));
   SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), at<float>(d, L.kbs),
                            st));
   SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<float>(d, L.kbs), wq, wk, at<float>(d, L.A),
@@ -237,7 +240,7 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
   o.status = desc->status;
   o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
-  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, Htot_out, Ztot_out, at<float>(desc, L.zscale), st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, nullptr, Htot_out, Ztot_out, nullptr, nullptr, st));
   return SLA2_OK;
 }
 
@@ -273,7 +276,7 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
 
   LinearOut o{};
   o.h = at<void>(desc, L.h);
-  o.h_mode = 1;
+  o.h_mode = 2;
   o.z = at<float>(desc, L.z);
   o.hpart = at<float>(desc, L.hpart);
   o.zpart = at<float>(desc, L.zpart);
@@ -286,8 +289,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   o.status = desc->status;
   o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
-  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
-                                at<float>(desc, L.zscale), st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, o.vamax, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
+                                at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), st));
   SLA2_TRY(mark(2));
 
   // sparse branch: tensor maps over the (quantised) operands
@@ -314,11 +317,10 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
 
   EpilogueArgs ea{};
   ea.q = q;
-  ea.Htot = at<float>(desc, L.Htot);
-  ea.Ztot = at<float>(desc, L.Ztot);
-  ea.zscale = at<float>(desc, L.zscale);
+  ea.htile = at<uint16_t>(desc, L.htile);
   ea.hT = at<uint16_t>(desc, L.h);
-  ea.z = o.z;
+  ea.hscale = at<float>(desc, L.hscale);
+  ea.Zi = at<float>(desc, L.Zi);
   ea.idx = idx;
   ea.os = os;
   ea.alpha = alpha;
@@ -328,10 +330,8 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  CUtensorMap tqe;
-  if (!make_map(&tqe, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B))
-    return SLA2_ERR_CUDA;
-  SLA2_TRY(launch_epilogue(s, ea, tqe, st));
+  if (s.k < s.nk) SLA2_TRY(launch_zsel(s, at<float>(desc, L.Ztot), o.z, idx, at<float>(desc, L.Zi), st));
+  SLA2_TRY(launch_epilogue(s, ea, st));
   SLA2_TRY(mark(4));
 
   // debug exports

@@ -168,6 +168,16 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] x B[smem]^T: A (M = 128 lanes, K packed two 16-bit
+// values per 32-bit column) read from tensor memory, B by descriptor.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 
 __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -231,6 +241,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       SLA2_W8(0), SLA2_W8(8), SLA2_W8(16), SLA2_W8(24)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      SLA2_W8(0), SLA2_W8(8)
       : "memory");
 }
 #undef SLA2_W8
@@ -297,6 +314,37 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Byte offset of the 16-byte chunk holding elements (row, col..col+7) of a
+// K-major 16-bit operand stored as 128-byte-swizzled slabs of 64 columns;
+// `slab_bytes` = rows * 128.
+__device__ __forceinline__ uint32_t sw128_h(int row, int col, int slab_bytes) {
+  return (uint32_t)((col >> 6) * slab_bytes + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+// Byte offset of the 16-byte chunk holding elements (row, col..col+7) of a
+// K-major 16-bit operand tile of `slabs` x 64 columns stored atom by atom:
+// each 8-row x 128-byte atom is 128-byte-swizzled, the slabs of one 8-row
+// group are adjacent (1024 bytes apart) and 8-row groups are slabs * 1024
+// bytes apart (the descriptor's stride byte offset). Tiles stored back to
+// back in this layout form one operand with more rows.
+__device__ __forceinline__ uint32_t atom_off(int row, int col, int slabs) {
+  return (uint32_t)((row >> 3) * (slabs * 1024) + (col >> 6) * 1024 + (row & 7) * 128 +
+                    ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+// Power of two s that keeps s * H_total (|H_total| <= N * max|V|, since every
+// phi entry is at most 1) at or below 2^15, inside the fp16 range, while the
+// per-block h_j (64 tokens) scaled the same way stay far above the fp16
+// subnormals. Identical on every CTA that evaluates it for the same inputs.
+__device__ __forceinline__ float h_fp16_scale(float vabs_max, int N) {
+  const float x = (float)N * vabs_max;
+  if (!(x > 0.f)) return 1.f;
+  int e = 141;
+  if (x < 3.0e38f) frexpf(x, &e);   // x = f * 2^e, f in [0.5, 1): x < 2^e
+  e = e < -112 ? -112 : (e > 141 ? 141 : e);
+  return ldexpf(1.f, 15 - e);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

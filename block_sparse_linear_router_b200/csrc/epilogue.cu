@@ -5,22 +5,41 @@
 //   O   = alpha_i O_s + (1 - alpha_i) O_l
 // When every key block is selected there is no unselected block and O_l := 0.
 //
+// The numerator never forms H_i: by linearity it is one tensor-core
+// accumulation over k + 1 operand tiles,
+//   D = phi(Q_i) (s H_total) + sum_{j selected} phi(Q_i) (-s h_j)
+// where the linear-state pass stored each -s h_j^T, and the reduce pass
+// s H_total^T, as fp16 d x d tiles already in the 128-byte-swizzled K-major
+// operand layout; s is a per-head power of two that keeps s H_total inside
+// the fp16 range. The denominator phi(Q_i) Z_i is a d-term fp32 dot product
+// per query row, taken while phi is computed; s cancels in O_l = D / (s den).
+//
+// The tiles go to the tensor core in groups of G = 256 / d, stacked along N,
+// so that every MMA is 128 x 256 x 16: at that size the tensor pipe hides the
+// per-group barrier wait and commit, which cost a large share of the time of
+// 128 x 128 MMAs. The accumulator then holds G column blocks, one per tile
+// slot, which the readout adds up.
+//
 // Persistent CTAs (one per SM) walk the (head, query block) items in
 // head-major order, so the SMs work on neighbouring query blocks of the same
-// head and the head's h_j^T stay in L2. Per CTA:
-//   warp 8     producer: per item, the bf16 Q tile by TMA (128-byte swizzle,
-//              the K-major operand layout) into one of two tile buffers, then
-//              the selected bf16 h_j^T tiles (contiguous d x d blocks) into a
-//              ring of shared-memory stages with 1-D bulk copies; it runs
-//              ahead of the compute warps across items;
-//   warps 0-7  per item: phi(Q_i) computed in place over the Q tile (fp16);
-//              H_i^T = H_total^T - sum of the ring tiles in fp32 registers;
-//              [H_i | Z_i] scaled by a per-head power of two (fp16 range) and
-//              written as the K-major B operand; one tcgen05 kind::f16 MMA
-//              chain D = phi(Q_i) [H_i | Z_i] (128 x (d+16) fp32 in TMEM:
-//              numerator columns 0..d-1, denominator column d); then
-//              O_l = num / den (the scale cancels), the alpha mix with O_s
-//              and the store.
+// head and the head's tiles stay in L2. Per CTA:
+//   warps 8,10 producers: each group's tiles, one 1-D bulk copy per tile,
+//              into a ring of shared-memory stages (a single issuing thread
+//              serialises its bulk copies, so two warps share the issue);
+//   warp 9     MMA issuer: per group, d/16 tcgen05 kind::f16 MMAs with
+//              A = phi(Q_i) in tensor memory and B = the stacked tiles, into
+//              the TMEM accumulator, then a commit that frees the stage;
+//   warps 0-7  per item: phi(Q_i), one query row
+//              per thread and half of the features per warp (the two halves
+//              exchange their row max and sum), stored as fp16 into one of two
+//              TMEM A buffers; the denominators phi(Q_i) . Z_i (Z_i precomputed
+//              per query block, copied in by producer 0); then, while the MMAs of this
+//              item run, the readout of the previous item: the accumulator is
+//              read into registers and released at once, then O_l = D / (s den),
+//              the alpha mix with O_s and the store.
+// A lives in tensor memory and Q / O_s go through registers, so shared memory
+// holds only the tile ring and its bandwidth goes to the tiles, each written
+// once by its copy and read once by the MMAs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -32,27 +51,30 @@ namespace sla2 {
 namespace {
 
 constexpr int EPI_COMPUTE = 256;          // warps 0-7
-constexpr int EPI_THREADS = EPI_COMPUTE + 32;
+constexpr int EPI_PRODUCER_WARP0 = 8;
+constexpr int EPI_MMA_WARP = 9;
+constexpr int EPI_PRODUCER_WARP1 = 10;
+constexpr int EPI_NPROD = 2;
+constexpr int EPI_THREADS = EPI_COMPUTE + 96;
 
 template <int D>
 struct EpiCfg {
-  static constexpr int NB = D + 16;                  // B rows (MMA N): H_i^T, Z_i, zeros
+  static constexpr int G = 256 / D;                  // tiles per group (MMA N = 256)
   static constexpr int SLABS = D / 64;               // K slabs of 64 fp16 (128 bytes)
-  static constexpr int QA_SLAB = BQ * 128;
-  static constexpr int QA_BYTES = SLABS * QA_SLAB;   // Q tile (bf16) -> phi (fp16), in place
-  static constexpr int B_SLAB = NB * 128;
-  static constexpr int B_BYTES = SLABS * B_SLAB;
-  static constexpr int TILE = D * D * 2;             // one bf16 h_j^T tile
-  static constexpr int NS = D == 128 ? 3 : 8;        // ring stages
-  static constexpr int OFF_B = 2 * QA_BYTES;
-  static constexpr int OFF_RING = OFF_B + B_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + NS * TILE;
-  static constexpr int NBAR = 2 * NS + 5;
+  static constexpr int TILE = D * D * 2;             // one fp16 operand tile (atom_off layout)
+  static constexpr int SBO = SLABS * 1024;           // bytes between 8-row groups of a tile / group
+  static constexpr int STAGE = G * TILE;             // one ring stage (a group: tiles back to back)
+  static constexpr int NS = (192 * 1024) / STAGE;    // ring stages: 3 (d = 128), 6 (d = 64)
+  static constexpr int HC = D / 2;                   // features (and output columns) per thread
+  static constexpr int OFF_Z = NS * STAGE;                    // Z_i of two items [2][D]
+  static constexpr int OFF_XCH = OFF_Z + 2 * D * 4;           // (max, sum) per row and half [2][BQ]
+  static constexpr int OFF_DEN = OFF_XCH + 2 * BQ * 8;        // denominator halves [2 buffers][2][BQ]
+  static constexpr int OFF_BAR = OFF_DEN + 4 * BQ * 4;
+  static constexpr int NBAR = 2 * NS + 9;
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
-  static constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, NB);   // fp16 x fp16 -> fp32
-  static constexpr int KSTEPS = D / 16;              // 16 fp16 (32 bytes) per MMA
-  static constexpr uint32_t TMEM_COLS = NB <= 128 ? 128 : 256;
-  static constexpr int SLOTS = D * D / 8 / EPI_COMPUTE;   // 8-element slots per compute thread
+  static constexpr int KSTEPS = D / 16;              // 16 fp16 (8 TMEM columns of A) per MMA
+  static constexpr uint32_t ACOL = 256;              // A buffers: columns ACOL + b * D / 2
+  static constexpr uint32_t TMEM_COLS = 512;
 };
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
@@ -67,11 +89,22 @@ __device__ __forceinline__ uint32_t h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Byte offset of the 16-byte chunk holding elements (row, col..col+7) of a
-// K-major 16-bit operand stored as 128-byte-swizzled slabs of 64 columns.
-__device__ __forceinline__ uint32_t sw128_h(int row, int col, int slab_bytes) {
-  return (uint32_t)((col >> 6) * slab_bytes + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+// Read-only 16-byte load kept where it is written (its latency overlaps the
+// work in between instead of being moved down to the first use).
+__device__ __forceinline__ uint4 ldg_v4_early(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(reinterpret_cast<uint64_t>(p)));
+  return r;
 }
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+// Barrier over the 256 compute threads.
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Barrier over the 256 compute threads that also returns, to every one of
 // them, whether any of them passed `failed` (so all take the same exit).
@@ -86,36 +119,76 @@ __device__ __forceinline__ bool compute_sync_any(bool failed) {
   return r != 0;
 }
 
+// O = alpha O_s + (1 - alpha) O_l for 32 consecutive columns of one row.
+__device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, float alpha, const float4* osv,
+                                          const float* ol) {
+  float o[32];
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 v = osv[c / 4];
+    o[c] = alpha * v.x + (1.f - alpha) * ol[c];
+    o[c + 1] = alpha * v.y + (1.f - alpha) * ol[c + 1];
+    o[c + 2] = alpha * v.z + (1.f - alpha) * ol[c + 2];
+    o[c + 3] = alpha * v.w + (1.f - alpha) * ol[c + 3];
+  }
+  if (a.ol_dbg) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4)
+      *reinterpret_cast<float4*>(a.ol_dbg + off + c) = make_float4(ol[c], ol[c + 1], ol[c + 2], ol[c + 3]);
+  }
+  if (a.out_f32) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4)
+      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + off + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + off;
+#pragma unroll
+    for (int c = 0; c < 32; c += 8)
+      *reinterpret_cast<uint4*>(dst + c) = make_uint4(cvt_bf16x2(o[c], o[c + 1]), cvt_bf16x2(o[c + 2], o[c + 3]),
+                                                      cvt_bf16x2(o[c + 4], o[c + 5]), cvt_bf16x2(o[c + 6], o[c + 7]));
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_constant__ CUtensorMap tq, Shape s,
-                                                                  EpilogueArgs a) {
+__global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, EpilogueArgs a) {
   using C = EpiCfg<D>;
   extern __shared__ uint8_t esm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sB = base + C::OFF_B;
-  uint8_t* ring = base + C::OFF_RING;
+  uint8_t* ring = base;
+  float* zbuf = reinterpret_cast<float*>(base + C::OFF_Z);
+  float2* xch = reinterpret_cast<float2*>(base + C::OFF_XCH);
+  float* den_s = reinterpret_cast<float*>(base + C::OFF_DEN);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
   uint64_t* empty = full + C::NS;
-  uint64_t* qfull = empty + C::NS;        // [2]
-  uint64_t* qfree = qfull + 2;            // [2]
-  uint64_t* mma_done = qfree + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  int* abort_flag = reinterpret_cast<int*>(mma_done + 1) + 1;
+  uint64_t* aready = empty + C::NS;       // [2] phi(Q) operand written to TMEM
+  uint64_t* dfull = aready + 2;           // accumulator complete
+  uint64_t* dfree = dfull + 1;            // accumulator read into registers
+  uint64_t* zfull = dfree + 1;            // [2] Z_i of an item landed
+  uint64_t* zfree = zfull + 2;            // [2] Z_i of an item used
+  uint64_t* drain = zfree + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* abort_flag = reinterpret_cast<int*>(drain + 1) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = s.BH * s.nq;
   const bool has_linear = s.k < s.nk;
+  const int ntile = s.k + 1;
+  const int nblk = ntile < C::G ? ntile : C::G;   // accumulator column blocks in use
 
   if (tid == 0) {
     for (int i = 0; i < C::NS; ++i) {
-      mbar_init(full + i, 1);
-      mbar_init(empty + i, EPI_COMPUTE);
+      mbar_init(full + i, EPI_NPROD);
+      mbar_init(empty + i, 1);
     }
+    mbar_init(aready, EPI_COMPUTE);
+    mbar_init(aready + 1, EPI_COMPUTE);
+    mbar_init(dfull, 1);
+    mbar_init(dfree, EPI_COMPUTE);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(qfull + b, 1);
-      mbar_init(qfree + b, 1);
+      mbar_init(zfull + b, 1);
+      mbar_init(zfree + b, EPI_COMPUTE);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,225 +196,262 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  // rows d+1 .. d+15 of the B operand are zero for every item
-  if (tid < EPI_COMPUTE) {
-    for (int t = tid; t < 15 * D / 8; t += EPI_COMPUTE)
-      *reinterpret_cast<uint4*>(sB + sw128_h(D + 1 + t / (D / 8), (t % (D / 8)) * 8, C::B_SLAB)) =
-          make_uint4(0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ---------------------------------------------------------------- producer
+  if (warp == EPI_PRODUCER_WARP0 || warp == EPI_PRODUCER_WARP1) {
+    // ---------------------------------------------------------------- producers
+    const int pr = warp == EPI_PRODUCER_WARP0 ? 0 : 1;   // this producer's tiles: t = pr, pr + 2, ...
     if (lane == 0 && has_linear) {
-      tma_prefetch_desc(&tq);
-      int g = 0, it = 0;
+      const size_t tile_elems = (size_t)D * D;
+      int st = 0, ng = 0, it = 0, nz = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
         const int bh = w / s.nq, qi = w % s.nq;
-        const int b = it & 1;
-        if (it >= 2 && !mbar_wait(qfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(qfull + b, C::QA_BYTES);
-#pragma unroll
-        for (int sl = 0; sl < C::SLABS; ++sl)
-          tma_load_2d(base + b * C::QA_BYTES + sl * C::QA_SLAB, &tq, qfull + b, sl * 64, bh * s.N + qi * BQ);
         const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * s.k;
-        for (int n = 0; n < s.k; ++n, ++g) {
-          const int st = g % C::NS;
-          if (g >= C::NS && !mbar_wait(empty + st, ((g / C::NS) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
+        if (pr == 0) {   // Z_i of this item (its buffer was last read for item it - 2)
+          const int b = it & 1;
+          if (it >= 2 && !mbar_wait(zfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
             ok = false;
             break;
           }
-          const int j = __ldg(sel + n);
-          mbar_arrive_expect_tx(full + st, C::TILE);
-          bulk_load(ring + st * C::TILE, a.hT + ((size_t)bh * s.nk + j) * D * D, C::TILE, full + st);
+          mbar_arrive_expect_tx(zfull + b, D * 4);
+          bulk_load(zbuf + b * D, a.Zi + ((size_t)bh * s.nq + qi) * D, D * 4, zfull + b);
+          ++nz;
+        }
+        for (int n0 = 0; n0 < ntile; n0 += C::G) {
+          const int cnt = ntile - n0 < C::G ? ntile - n0 : C::G;
+          if (ng >= C::NS && !mbar_wait(empty + st, ph ^ 1u, abort_flag, a.status, a.budget_ns)) {
+            ok = false;
+            break;
+          }
+          const int mine = cnt > pr ? (cnt - pr + EPI_NPROD - 1) / EPI_NPROD : 0;
+          mbar_arrive_expect_tx(full + st, (uint32_t)(mine * C::TILE));
+          uint8_t* dst = ring + st * C::STAGE;
+          for (int t = pr; t < cnt; t += EPI_NPROD) {
+            const int n = n0 + t;
+            const uint16_t* src = n == 0 ? a.htile + (size_t)bh * tile_elems
+                                         : a.hT + ((size_t)bh * s.nk + __ldg(sel + n - 1)) * tile_elems;
+            bulk_load(dst + t * C::TILE, src, C::TILE, full + st);
+          }
+          ++ng;
+          if (++st == C::NS) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
       }
       if (!ok) {   // let the copies in flight land before the CTA's shared memory is released
-        for (int q = (g > C::NS ? g - C::NS : 0); q < g; ++q)
+        for (int q = (ng > C::NS ? ng - C::NS : 0); q < ng; ++q)
           mbar_wait_drain(full + q % C::NS, (q / C::NS) & 1, 20000000ull);
-        for (int q = (it > 2 ? it - 2 : 0); q <= it; ++q) mbar_wait_drain(qfull + (q & 1), (q >> 1) & 1, 20000000ull);
+        for (int q = (nz > 2 ? nz - 2 : 0); q < nz; ++q) mbar_wait_drain(zfull + (q & 1), (q >> 1) & 1, 20000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == EPI_MMA_WARP) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && has_linear) {
+      const uint64_t bdesc0 = make_sdesc(smem_u32(ring), C::SBO, LAYOUT_SW128);
+      int st = 0, it = 0;
+      uint32_t ph = 0;
+      bool ok = true, issued = false;
+      for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
+        const int b = it & 1;
+        if (!mbar_wait(aready + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
+        if (it >= 1 && !mbar_wait(dfree, (it - 1) & 1, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t acol = tmem + C::ACOL + (uint32_t)(b * (D / 2));
+        for (int n0 = 0; n0 < ntile; n0 += C::G) {
+          const int cnt = ntile - n0 < C::G ? ntile - n0 : C::G;
+          const uint32_t idesc = make_idesc(1, 0, 0, 128, (uint32_t)(cnt * D));   // fp16 x fp16 -> fp32
+          if (!mbar_wait(full + st, ph, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
+          tc_fence_after();
+          // descriptor start addresses advance in 16-byte units
+          const uint64_t bd = bdesc0 + (uint64_t)((st * C::STAGE) >> 4);
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS; ++ks)
+            mma_f16_ts(tmem, acol + ks * 8, bd + (uint64_t)(((ks >> 2) * 1024 + (ks & 3) * 32) >> 4), idesc,
+                       (n0 | ks) != 0);
+          issued = true;
+          tc_commit(empty + st);
+          if (++st == C::NS) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(dfull);
+      }
+      if (!ok && issued) {   // issued MMAs finish before the CTA releases TMEM and shared memory
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, 20000000ull);
       }
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warps
-    constexpr int TPR = D / 8, RPP = EPI_COMPUTE / TPR;
-    const int cg = tid % TPR, rg = tid / TPR;
-    const int r = (warp & 3) * 32 + lane;        // TMEM lane / query row of the readout
-    const int half = warp >> 2;
-    constexpr int HC = D / 2;
-    const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    int g = 0, it = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-      const int bh = w / s.nq, qi = w % s.nq;
-      const int h = bh % a.H;
-      const float alpha = a.alpha[(size_t)h * s.nq + qi];
-      const size_t row = (size_t)bh * s.N + (size_t)qi * BQ + r;
-      float4 osv[HC / 4];
-      if (has_linear) {
-        const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * s.k;
-        uint8_t* qa = base + (it & 1) * C::QA_BYTES;
-        // ---- H_total^T (issued first; its loads overlap the phi work)
-        float acc[C::SLOTS][8];
-        const float4* Ht = reinterpret_cast<const float4*>(a.Htot + (size_t)bh * D * D);
+    constexpr int HC = C::HC;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const int qd = warp & 3, fh = warp >> 2;     // TMEM lane quadrant, feature / column half
+    const int r = qd * 32 + lane;                // query row of the block = TMEM lane
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    auto row_of = [&](int w) { return (size_t)(w / s.nq) * s.N + (size_t)(w % s.nq) * BQ + r; };
+
+    if (!has_linear) {
+      float zero[32];
 #pragma unroll
-        for (int u = 0; u < C::SLOTS; ++u) {
-          const int slot = tid + u * EPI_COMPUTE;
-          const float4 x0 = __ldg(Ht + 2 * slot), x1 = __ldg(Ht + 2 * slot + 1);
-          acc[u][0] = x0.x; acc[u][1] = x0.y; acc[u][2] = x0.z; acc[u][3] = x0.w;
-          acc[u][4] = x1.x; acc[u][5] = x1.y; acc[u][6] = x1.z; acc[u][7] = x1.w;
+      for (int c = 0; c < 32; ++c) zero[c] = 0.f;
+      for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        const int bh = w / s.nq, qi = w % s.nq;
+        const float alpha = a.alpha[(size_t)(bh % a.H) * s.nq + qi];
+        const size_t row = row_of(w);
+#pragma unroll
+        for (int cc = 0; cc < HC / 32; ++cc) {
+          float4 osv[8];
+          const float4* osr = reinterpret_cast<const float4*>(a.os + row * D + fh * HC + cc * 32);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) osv[c] = __ldg(osr + c);
+          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, zero);
         }
-        // ---- phi(Q_i) in place over the TMA-loaded bf16 Q tile -> fp16
-        ok = mbar_wait(qfull + (it & 1), (it >> 1) & 1, abort_flag, a.status, a.budget_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-#pragma unroll 2
-          for (int rr = rg; rr < BQ; rr += RPP) {
-            uint4* p = reinterpret_cast<uint4*>(qa + sw128_h(rr, cg * 8, C::QA_SLAB));
-            float x[8];
-            unpack8(*p, x);
-            float m = x[0];
+      }
+    } else {
+      // readout of item `itp` (work index wp): the accumulator's column blocks
+      // summed into registers, the accumulator released, then O_l, mix, store
+      auto readout = [&](int itp, int wp) -> bool {
+        const int bh = wp / s.nq, qi = wp % s.nq;
+        const float alpha = a.alpha[(size_t)(bh % a.H) * s.nq + qi];
+        const float hsc = a.hscale[bh];
+        const size_t row = row_of(wp);
+        const int bp = itp & 1;
+        const float* osr = a.os + row * D + fh * HC;
+        float4 osv[8];
 #pragma unroll
-            for (int c = 1; c < 8; ++c) m = fmaxf(m, x[c]);
-#pragma unroll
-            for (int off = TPR / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              x[c] = expf(x[c] - m);
-              sum += x[c];
-            }
-#pragma unroll
-            for (int off = TPR / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            const float inv = 1.f / sum;
-            *p = make_uint4(h2(x[0] * inv, x[1] * inv), h2(x[2] * inv, x[3] * inv), h2(x[4] * inv, x[5] * inv),
-                            h2(x[6] * inv, x[7] * inv));
-          }
-        }
-        // ---- H_i^T = H_total^T - sum of the selected h_j^T
-        for (int n = 0; ok && n < s.k; ++n, ++g) {
-          const int st = g % C::NS;
-          ok = mbar_wait(full + st, (g / C::NS) & 1, abort_flag, a.status, a.budget_ns);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          const uint4* tile = reinterpret_cast<const uint4*>(ring + st * C::TILE);
-#pragma unroll
-          for (int u = 0; u < C::SLOTS; ++u) {
-            float x[8];
-            unpack8(tile[tid + u * EPI_COMPUTE], x);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[u][c] -= x[c];
-          }
-          mbar_arrive(empty + st);
-        }
-        // ---- [H_i^T ; Z_i] * scale -> fp16 B operand
-        const float sc = a.zscale[bh];
-#pragma unroll
-        for (int u = 0; u < C::SLOTS; ++u) {
-          const int slot = tid + u * EPI_COMPUTE;
-          const int brow = slot / (D / 8), bcol = (slot % (D / 8)) * 8;
-          *reinterpret_cast<uint4*>(sB + sw128_h(brow, bcol, C::B_SLAB)) =
-              make_uint4(h2(acc[u][0] * sc, acc[u][1] * sc), h2(acc[u][2] * sc, acc[u][3] * sc),
-                         h2(acc[u][4] * sc, acc[u][5] * sc), h2(acc[u][6] * sc, acc[u][7] * sc));
-        }
-        if (tid < D / 8) {
-          float z[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) z[c] = a.Ztot[(size_t)bh * D + tid * 8 + c];
-          for (int n = 0; n < s.k; ++n) {
-            const float* zj = a.z + ((size_t)bh * s.nk + __ldg(sel + n)) * D + tid * 8;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) z[c] -= zj[c];
-          }
-          *reinterpret_cast<uint4*>(sB + sw128_h(D, tid * 8, C::B_SLAB)) =
-              make_uint4(h2(z[0] * sc, z[1] * sc), h2(z[2] * sc, z[3] * sc), h2(z[4] * sc, z[5] * sc),
-                         h2(z[6] * sc, z[7] * sc));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (compute_sync_any(!ok)) break;     // every compute thread takes this exit together
-        // ---- D = phi(Q_i) [H_i | Z_i]
-        if (tid == 0) {
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(qa), b0 = smem_u32(sB);
-#pragma unroll
-          for (int ks = 0; ks < C::KSTEPS; ++ks) {
-            const uint32_t off = (ks & 3) * 32;
-            const uint64_t ad = make_sdesc(a0 + (ks >> 2) * C::QA_SLAB + off, 1024, LAYOUT_SW128);
-            const uint64_t bd = make_sdesc(b0 + (ks >> 2) * C::B_SLAB + off, 1024, LAYOUT_SW128);
-            mma_f16(tmem, ad, bd, C::IDESC, ks > 0);
-          }
-          tc_commit(mma_done);
-          tc_commit(qfree + (it & 1));
-        }
-        // O_s loads overlap the MMA
-        const float* osr = a.os + row * D + half * HC;
-#pragma unroll
-        for (int c = 0; c < HC / 4; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr) + c);
-        ok = mbar_wait(mma_done, it & 1, abort_flag, a.status, a.budget_ns);
+        for (int c = 0; c < 8; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr) + c);
+        bool ok = mbar_wait(dfull, itp & 1, abort_flag, a.status, a.budget_ns);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
-        if (!ok) continue;   // a failed wait: skip the store; the next barrier ends the loop
-      } else {
-        const float* osr = a.os + row * D + half * HC;
+        if (!ok) return false;
+        float ol[HC];
 #pragma unroll
-        for (int c = 0; c < HC / 4; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr) + c);
-      }
-      // ---- O_l, mix, store: warp w reads TMEM lanes 32 (w % 4).., column half w / 4
-      float inv_den = 0.f;
-      if (has_linear) {
-        uint32_t dv[32];
-        tmem_ld32(taddr + D, dv);
-        tmem_wait_ld();
-        inv_den = 1.f / __uint_as_float(dv[0]);
-      }
-#pragma unroll
-      for (int cc = 0; cc < HC / 32; ++cc) {
-        uint32_t nv[32];
-        if (has_linear) {
-          tmem_ld32(taddr + half * HC + cc * 32, nv);
+        for (int cc = 0; cc < HC / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)(fh * HC + cc * 32), v);
           tmem_wait_ld();
-        }
-        float o[32], ol[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          const float4 v = osv[(cc * 32 + c) / 4];
-          const float os4[4] = {v.x, v.y, v.z, v.w};
+          for (int c = 0; c < 32; ++c) ol[cc * 32 + c] = __uint_as_float(v[c]);
+          for (int blk = 1; blk < nblk; ++blk) {
+            tmem_ld32(tmem + lane_base + (uint32_t)(blk * D + fh * HC + cc * 32), v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            ol[c + u] = has_linear ? __uint_as_float(nv[c + u]) * inv_den : 0.f;
-            o[c + u] = alpha * os4[u] + (1.f - alpha) * ol[c + u];
+            for (int c = 0; c < 32; ++c) ol[cc * 32 + c] += __uint_as_float(v[c]);
           }
         }
-        const size_t off = row * D + half * HC + cc * 32;
-        if (a.ol_dbg) {
+        tc_fence_before();
+        mbar_arrive(dfree);
+        const float inv = 1.f / (hsc * (den_s[(bp * 2) * BQ + r] + den_s[(bp * 2 + 1) * BQ + r]));
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(a.ol_dbg + off + c) = make_float4(ol[c], ol[c + 1], ol[c + 2], ol[c + 3]);
+        for (int c = 0; c < HC; ++c) ol[c] *= inv;
+#pragma unroll
+        for (int cc = 0; cc < HC / 32; ++cc) {
+          if (cc > 0) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr + cc * 32) + c);
+          }
+          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, ol + cc * 32);
         }
-        if (a.out_f32) {
+        return true;
+      };
+
+      uint4 qv[HC / 8];                          // this thread's half row of Q (bf16)
+      auto load_q = [&](int w) {               // issued here, consumed one item later
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row_of(w) * D + fh * HC);
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(static_cast<float*>(a.out) + off + c) =
-                make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        for (int i = 0; i < HC / 8; ++i) qv[i] = ldg_v4_early(src + i);
+      };
+      load_q(blockIdx.x);
+      int it = 0, wprev = -1;
+      bool ok = true, rd_ok = true;
+      for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+        const int bh = w / s.nq, qi = w % s.nq;
+        const int b = it & 1;
+        if (wprev >= 0) {                        // O_s of the previous item, read out below
+          const float* p = a.os + row_of(wprev) * D + fh * HC;
+#pragma unroll
+          for (int c = 0; c < HC; c += 32) prefetch_l2(p + c);
+        }
+        (void)bh;
+        (void)qi;
+        // ---- phi = softmax over the d features: local max / sum, then exchanged between the halves
+        float x[HC];
+#pragma unroll
+        for (int q = 0; q < HC / 8; ++q) {
+          float v8[8];
+          unpack8(qv[q], v8);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) x[q * 8 + c] = v8[c];
+        }
+        {
+          const int wn = w + gridDim.x;          // the next item's Q rows, consumed next iteration
+          if (wn < total) load_q(wn);
+        }
+        // four independent partial chains for the max and the sum
+        float m4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int c = 4; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
+        const float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const float mb = m * kLog2e;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < HC; ++c) {
+          x[c] = ex2_approx(fmaf(x[c], kLog2e, -mb));
+          s4[c & 3] += x[c];
+        }
+        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        xch[fh * BQ + r] = make_float2(m, sum);
+        compute_sync();
+        const float2 o = xch[(fh ^ 1) * BQ + r];
+        const float M = fmaxf(m, o.x);
+        const float e_own = ex2_approx((m - M) * kLog2e);
+        const float scale = e_own / (sum * e_own + o.y * ex2_approx((o.x - M) * kLog2e));
+        // den = phi(Q_i) . Z_i over this half of the features
+        bool zok = mbar_wait(zfull + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns);
+        zok = __all_sync(0xffffffffu, zok);
+        ok = ok && zok;
+        const float4* zi4 = reinterpret_cast<const float4*>(zbuf + b * D + fh * HC);
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[HC / 2];
+#pragma unroll
+        for (int c = 0; c < HC; c += 4) {
+          const float4 zz = zok ? zi4[c / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float p0 = x[c] * scale, p1 = x[c + 1] * scale, p2 = x[c + 2] * scale, p3 = x[c + 3] * scale;
+          d4[0] = fmaf(p0, zz.x, d4[0]);
+          d4[1] = fmaf(p1, zz.y, d4[1]);
+          d4[2] = fmaf(p2, zz.z, d4[2]);
+          d4[3] = fmaf(p3, zz.w, d4[3]);
+          pk[c / 2] = h2(p0, p1);
+          pk[c / 2 + 1] = h2(p2, p3);
+        }
+        mbar_arrive(zfree + b);
+        den_s[(b * 2 + fh) * BQ + r] = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+        const uint32_t ta = tmem + lane_base + C::ACOL + (uint32_t)(b * (D / 2) + fh * (HC / 2));
+        if constexpr (HC / 2 == 32) {
+          tmem_st32(ta, pk);
         } else {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + off;
-#pragma unroll
-          for (int c = 0; c < 32; c += 8)
-            *reinterpret_cast<uint4*>(dst + c) =
-                make_uint4(cvt_bf16x2(o[c], o[c + 1]), cvt_bf16x2(o[c + 2], o[c + 3]),
-                           cvt_bf16x2(o[c + 4], o[c + 5]), cvt_bf16x2(o[c + 6], o[c + 7]));
+          tmem_st16(ta, pk);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(aready + b);
+        // every compute thread takes this exit together
+        if (compute_sync_any(!ok || !rd_ok)) { ok = false; break; }
+        // ---- the previous item's readout overlaps this item's MMAs
+        if (wprev >= 0) rd_ok = readout(it - 1, wprev);
+        wprev = w;
       }
-      tc_fence_before();
+      if (ok && rd_ok && wprev >= 0) readout(it - 1, wprev);
     }
   }
   tc_fence_before();
@@ -352,21 +462,39 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
   }
 }
 
+// Z_i = Z_total - sum of the selected z_j for every (head, query block), one
+// feature per thread, the selected blocks in ascending order.
+__global__ void zsel_kernel(const float* __restrict__ Ztot, const float* __restrict__ z, const int32_t* __restrict__ idx,
+                            int nq, int nk, int k, float* __restrict__ Zi) {
+  const int qi = blockIdx.x, bh = blockIdx.y, c = threadIdx.x, D = blockDim.x;
+  const int32_t* sel = idx + ((size_t)bh * nq + qi) * k;
+  float acc = Ztot[(size_t)bh * D + c];
+#pragma unroll 8
+  for (int n = 0; n < k; ++n) acc -= z[((size_t)bh * nk + __ldg(sel + n)) * D + c];
+  Zi[((size_t)bh * nq + qi) * D + c] = acc;
+}
+
 constexpr int kSMs = 148;   // B200 streaming multiprocessors
 
 }  // namespace
 
-cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, const CUtensorMap& tq, cudaStream_t st) {
+cudaError_t launch_zsel(const Shape& s, const float* Ztot, const float* z, const int32_t* idx, float* Zi,
+                        cudaStream_t st) {
+  zsel_kernel<<<dim3(s.nq, s.BH), s.d, 0, st>>>(Ztot, z, idx, s.nq, s.nk, s.k, Zi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st) {
   const int total = s.BH * s.nq;
   const int grid = total < kSMs ? total : kSMs;
   if (s.d == 128) {
     auto k = epilogue_kernel<128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<128>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(tq, s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(s, a);
   } else {
     auto k = epilogue_kernel<64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<64>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(tq, s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(s, a);
   }
   return cudaGetLastError();
 }

@@ -42,7 +42,12 @@ int scores_topk_max_nk();
 // Per key block: h_j, z_j (fp32) and per-chunk partial sums; optionally K-hat /
 // s_k and V-hat^T / s_v (quant = 1: e4m3; quant = 0: bf16 copy of V^T).
 struct LinearOut {
-  void* h;           // h_j^T [BH][nk][d (channel c)][d (feature e)]: h_mode 0 fp32, 1 bf16
+  // h_j^T [BH][nk][d (V channel e)][d (phi feature c)], by h_mode:
+  //   0: fp32 row-major;  1: bf16 row-major;
+  //   2: fp16 -s h_j^T (s = h_fp16_scale of the head, from vamax) as the image of
+  //      a K-major operand tile in the atom_off layout: 8-row x 128-byte atoms,
+  //      16-byte chunks swizzled by row & 7 (what the epilogue's MMA reads as B).
+  void* h;
   int h_mode;        // partial sums (and so H_total) are always written transposed too
   float* z;          // [BH][nk][d]
   float* hpart;      // [BH][G][d][d]
@@ -51,7 +56,7 @@ struct LinearOut {
   float* sk;         // [BH][nk]
   void* vhatT;       // [BH][nk][d][64] (u8 e4m3 or bf16) or nullptr
   float* sv;         // [BH][d]
-  const unsigned* vamax;  // [BH][d] (quant = 1)
+  const unsigned* vamax;  // [BH][d] per-channel max |V| as float bits (quant = 1 or h_mode = 2)
   int quant;
   unsigned* status;
   unsigned long long budget_ns;
@@ -60,8 +65,10 @@ struct LinearOut {
 int linear_chunks(int BH, int nk);
 cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, const float* c32, const LinearOut& o,
                                 cudaStream_t st);
-cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, float* Htot, float* Ztot,
-                                 float* zscale, cudaStream_t st);
+// H_total^T / Z_total (fp32) from the chunk partials; optionally (vamax given)
+// the fp16 image of s H_total^T in the h_mode-2 layout and s per head.
+cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, const unsigned* vamax,
+                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st);
 
 // ---- sparse branch (sparse.cu) --------------------------------------------
 struct SparseArgs {
@@ -80,22 +87,24 @@ size_t sparse_smem_bytes(int d, int quant);
 
 // ---- epilogue (epilogue.cu) -----------------------------------------------
 struct EpilogueArgs {
-  const void* q;        // bf16 [BH][N][d]
-  const float* Htot;    // H_total^T [BH][d][d] (fp32)
-  const float* Ztot;    // [BH][d]
-  const float* zscale;  // [BH] power of two with Z_total * zscale <= 1
-  const uint16_t* hT;   // h_j^T bf16 [BH][nk][d][d]
-  const float* z;       // [BH][nk][d]
-  const int32_t* idx;   // [BH][nq][k]
-  const float* os;      // [BH][N][d]
-  const float* alpha;   // [H][nq]
+  const void* q;          // bf16 [BH][N][d]
+  const uint16_t* htile;  // fp16 s H_total^T operand images [BH][d*d] (h_mode-2 layout)
+  const uint16_t* hT;     // fp16 -s h_j^T operand images [BH][nk][d*d] (h_mode 2)
+  const float* hscale;    // [BH] s
+  const float* Zi;        // [BH][nq][d] Z_total - sum of the selected z_j
+  const int32_t* idx;     // [BH][nq][k]
+  const float* os;        // [BH][N][d]
+  const float* alpha;     // [H][nq]
   int H;
-  void* out;            // [BH][N][d]
+  void* out;              // [BH][N][d]
   int out_f32;
-  float* ol_dbg;        // optional [BH][N][d]
+  float* ol_dbg;          // optional [BH][N][d]
   unsigned* status;
   unsigned long long budget_ns;
 };
-cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, const CUtensorMap& tq, cudaStream_t st);
+// Z_i per (head, query block), the epilogue's denominators' second factor
+cudaError_t launch_zsel(const Shape& s, const float* Ztot, const float* z, const int32_t* idx, float* Zi,
+                        cudaStream_t st);
+cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st);
 
 }  // namespace sla2

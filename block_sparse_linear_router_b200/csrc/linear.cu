@@ -13,6 +13,10 @@
 //   h_j^T = V_j^T phi_j  on the tensor core: tcgen05 kind::f16 with fp16
 //           operands (V exactly, phi rounded once), fp32 accumulation in TMEM;
 //           a second TMEM accumulator sums h_j^T over the chunk (partial H^T).
+//           h_j^T is stored as fp32 or bf16 rows, or (forward pass) as the
+//           fp16 tile -s h_j^T already in a swizzled K-major operand layout
+//           (atom by atom), which the epilogue's tensor-core MMA consumes as
+//           it lands.
 // The staged tiles are [token][column] with 128-byte swizzle, which is the
 // MN-major operand layout: the converters overwrite K with phi (fp16) and V
 // with V (fp16) in place, and the MMA reads them as A = V (M = channel) and
@@ -171,6 +175,16 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         for (int t = tid; t < C::SLAB / 16; t += 128)
           *reinterpret_cast<uint4*>(base + st * C::STAGE + C::OFF_V + C::KV_TILE + t * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
+    float hs = 1.f;                  // h_mode 2: the head's fp16 operand scale
+    if (o.h_mode == 2) {
+      float m = tid < D ? __uint_as_float(o.vamax[(size_t)bh * D + tid]) : 0.f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (lane == 0) zred_all[warp] = m;
+      conv_sync();
+      hs = h_fp16_scale(fmaxf(fmaxf(zred_all[0], zred_all[1]), fmaxf(zred_all[2], zred_all[3])), N);
+      conv_sync();
+    }
     float zp = 0.f;                  // this thread's feature (tid < D) partial of Z
     const uint32_t lane_taddr = tmem + ((uint32_t)(warp * 32) << 16);
     bool ok = true;
@@ -314,7 +328,17 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
           uint32_t r[32];
           tmem_ld32(lane_taddr + cc * 32, r);
           tmem_wait_ld();
-          if (o.h_mode == 1) {
+          if (o.h_mode == 2) {
+            uint8_t* tile = static_cast<uint8_t*>(o.h) + ((size_t)bh * nk + j) * (size_t)(D * D * 2);
+            const float ns = -hs;
+#pragma unroll
+            for (int q = 0; q < 32; q += 8)
+              *reinterpret_cast<uint4*>(tile + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
+                  h2_bits(ns * __uint_as_float(r[q]), ns * __uint_as_float(r[q + 1])),
+                  h2_bits(ns * __uint_as_float(r[q + 2]), ns * __uint_as_float(r[q + 3])),
+                  h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
+                  h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
+          } else if (o.h_mode == 1) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
 #pragma unroll
             for (int q = 0; q < 32; q += 8)
@@ -359,39 +383,44 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   }
 }
 
-// H_total^T and Z_total as fixed-order sums of the chunk partials, plus a
-// per-head power of two 2^-E >= ... with max_e Z_total[e] <= 2^E, which the
-// epilogue applies to H_i and Z_i so that both fit fp16 operands exactly
-// scaled (the ratio H_i / Z_i does not change).
+// H_total^T and Z_total as fixed-order sums of the chunk partials. With vamax
+// given, also the head's fp16 scale s (the same value the linear-state pass
+// used for its h_j tiles) and s H_total^T as an fp16 operand image in the
+// h_mode-2 layout, which the epilogue loads as the first B tile of every item.
 __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const float* __restrict__ zpart, int G, int D,
-                                     float* __restrict__ Htot, float* __restrict__ Ztot, float* __restrict__ zscale) {
-  __shared__ float zmax[8];
+                                     int N, const unsigned* __restrict__ vamax, float* __restrict__ Htot,
+                                     float* __restrict__ Ztot, uint16_t* __restrict__ htile,
+                                     float* __restrict__ hscale) {
+  __shared__ float red[8];
   const int bh = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   const int DD = D * D;
+  float hs = 1.f;
+  if (vamax) {
+    float m = threadIdx.x < D ? __uint_as_float(vamax[(size_t)bh * D + threadIdx.x]) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    float mx = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, red[w]);
+    hs = h_fp16_scale(mx, N);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && hscale) hscale[bh] = hs;
+  }
   if (e < DD) {
     float s = 0.f;
     for (int g = 0; g < G; ++g) s += hpart[((size_t)bh * G + g) * DD + e];
     Htot[(size_t)bh * DD + e] = s;
+    if (vamax && htile) {
+      const int row = e / D, col = e % D;
+      const __half hv = __float2half_rn(hs * s);
+      htile[(size_t)bh * DD + (atom_off(row, col, D / 64) >> 1) + (col & 7)] = *reinterpret_cast<const uint16_t*>(&hv);
+    }
   }
-  if (blockIdx.x == 0) {
+  if (blockIdx.x == 0 && threadIdx.x < D) {
     float s = 0.f;
-    if (threadIdx.x < D) {
-      for (int g = 0; g < G; ++g) s += zpart[((size_t)bh * G + g) * D + threadIdx.x];
-      Ztot[(size_t)bh * D + threadIdx.x] = s;
-    }
-    float m = s;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) zmax[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0 && zscale) {
-      float mx = 0.f;
-      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, zmax[w]);
-      int ex = 0;
-      frexpf(mx, &ex);                       // mx = f * 2^ex, f in [0.5, 1)
-      zscale[bh] = mx > 0.f ? ldexpf(1.f, -ex) : 1.f;
-    }
+    for (int g = 0; g < G; ++g) s += zpart[((size_t)bh * G + g) * D + threadIdx.x];
+    Ztot[(size_t)bh * D + threadIdx.x] = s;
   }
 }
 
@@ -425,11 +454,12 @@ cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, co
   return cudaGetLastError();
 }
 
-cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, float* Htot, float* Ztot,
-                                 float* zscale, cudaStream_t st) {
+cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, const unsigned* vamax,
+                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st) {
   const int DD = s.d * s.d;
   dim3 grid((DD + 255) / 256, s.BH);
-  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, Htot, Ztot, zscale);
+  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, s.N, vamax, Htot, Ztot,
+                                             htile, hscale);
   return cudaGetLastError();
 }
 
