@@ -63,7 +63,38 @@ def work_model(w, k):
         # repeated tile gather (k + 1 per query block) is L2 traffic, reported separately
         "epilogue_bytes": 2 * E + 4 * E + 2 * E + BH * nk * d * d * 2,
         "gather_bytes": BH * nq * (k + 1) * d * d * 2,   # per query block: H_total and the k selected h_j tiles
+        # epilogue MMAs: phi(Q_i) (128 x d) times k + 1 tiles (d x d), fp16 in, fp32 accumulate
+        "epilogue_flops": BH * nq * (k + 1) * 2 * 128 * d * d if k < nk else 0,
     }
+
+
+# DRAM bytes per launch measured by ncu (summaries under profiles/), valid only for the
+# kernel source they were taken on: sha256 prefix of the kernel file + device.cuh + kernels.cuh.
+MEASURED_TRAFFIC = {
+    # dram__bytes_read.sum + dram__bytes_write.sum, --set full capture
+    "sparse": ("sparse.cu", "4a052642555b5e87", 298.0e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    # dram__bytes.sum.per_second x gpu__time_duration.sum, section capture
+    "epilogue": ("epilogue.cu", "cbefc15d0eb99f09", 594.0e6, "ncu dram__bytes.sum.per_second x duration"),
+    "linear_state": ("linear.cu", "5e42d52ed190c7af", 472.0e6, "ncu dram__bytes.sum.per_second x duration"),
+}
+
+
+def measured_traffic(name):
+    """(bytes, source) of the ncu capture for this stage's kernel, or (None, None) once the
+    kernel source differs from the one that was profiled."""
+    import hashlib
+    if name not in MEASURED_TRAFFIC:
+        return None, None
+    f, sha, b, src = MEASURED_TRAFFIC[name]
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_linear_router_b200", "csrc")
+    h = hashlib.sha256()
+    try:
+        for part in (f, "device.cuh", "kernels.cuh"):
+            with open(os.path.join(csrc, part), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None, None
+    return (b, src) if h.hexdigest()[:16] == sha else (None, None)
 
 
 def launches_per_forward(w, k):
@@ -329,20 +360,34 @@ def main():
     p8 = peaks["bf16_tflops"] * NOMINAL_8BIT_OVER_BF16
     names = ["router", "linear_state", "sparse", "epilogue"]
     kern = {}
+    p16 = peaks["bf16_tflops"]   # fp16 and bf16 run at the same dense rate
     for n, msv in zip(names, stage_ms):
         if n == "sparse":
             ach = wm["sparse_ops"] / (msv * 1e-3) / 1e12
             kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p8, "unit": "TOPS", "frac": ach / p8}
+        elif n == "epilogue" and wm["epilogue_flops"] > 0:
+            # tensor-bound when its MMA time exceeds its HBM time (206 GFLOP vs 604 MB here)
+            ach = wm["epilogue_flops"] / (msv * 1e-3) / 1e12
+            hb = wm["epilogue_bytes"] / (msv * 1e-3) / 1e9
+            kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p16, "unit": "TFLOP/s",
+                       "frac": ach / p16, "hbm_achieved_gbs": hb, "hbm_frac": hb / hbm,
+                       "algorithmic_bytes": wm["epilogue_bytes"], "flops": wm["epilogue_flops"]}
         else:
             b = wm[f"{n.split('_')[0]}_bytes"] if n != "linear_state" else wm["linear_bytes"]
             ach = b / (msv * 1e-3) / 1e9
             kern[n] = {"ms": msv, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                        "algorithmic_bytes": b}
+    for n in names:
+        tb, tsrc = measured_traffic(n)
+        kern[n]["traffic"] = tb
+        if tb is not None:
+            kern[n]["traffic_source"] = tsrc
     dom = max(names, key=lambda n: kern[n]["ms"])
     dk = kern[dom]
+    psrc = {"sparse": "8-bit = bf16 burst x 2 nominal ratio", "epilogue": "fp16 = bf16 burst (same dense rate)"}
     roofline = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
-                "frac": dk["frac"], "traffic": None, "kernel": dom,
-                "peak_source": f"{peak_src} ({'8-bit = bf16 burst x 2 nominal ratio' if dom == 'sparse' else 'HBM copy'})"}
+                "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dom,
+                "peak_source": f"{peak_src} ({psrc.get(dom, 'HBM copy') if dk['bound'] == 'tensor' else 'HBM copy'})"}
 
     cpu = None
     if not args.no_cpu_baseline:
