@@ -156,7 +156,12 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
 
 /* The whole forward pass (steps 1-4): out = alpha O_s + (1 - alpha) O_l.
  *   out : bf16 or fp32 (desc->out_dtype) [B][H][N][d]
- * All intermediates live in desc->workspace; optional debug exports in desc. */
+ * All intermediates live in desc->workspace; optional debug exports in desc.
+ * Arithmetic: router in fp32; sparse branch INT8 Q K^T (int32 accumulate) and
+ * e4m3 P V (fp32 accumulate) with quantize = 1, bf16 operands with quantize = 0;
+ * linear branch on fp16 tensor-core operands with fp32 accumulation, h_j and
+ * H_total scaled per head by a power of two derived from max|V| (V magnitudes
+ * up to about 1e30 stay in range). */
 sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v,
                          const float* proj_q, const float* proj_k, const float* alpha,
                          float topk_frac, void* out, void* stream);
