@@ -400,7 +400,11 @@ def main():
         "data": "synthetic",
         "config": {"workload": f"{w.name} B={w.B} H={w.H} N={w.N} d={w.d} k%={w.topk_frac * 100:g} (k={k} of {w.nk})",
                    "l2": "no flush: Q/K/V 302 MB > 126 MB L2", "parallelism": f"replicas x{ws}"},
-        "roofline": roofline, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "kernels": kern,
+        "stages": "router = pass over Q/K/V + column means; linear_state = linear state + reduce, with the "
+                  "router's projections / logits / top-k concurrent on a second stream; sparse = sparse branch "
+                  "(Z_i concurrent); epilogue = linear apply + mix",
+        "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_forward(w, k) * K, "clocks": clk,
         "sparse_issued_tops": kern["sparse"]["achieved"],
     }

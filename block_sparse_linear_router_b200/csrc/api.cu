@@ -152,9 +152,9 @@ sla2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA2_OK : SLA
     if (_e != cudaSuccess) return SLA2_ERR_CUDA;         \
   } while (0)
 
-sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
-                       const void* v, const float* wq, const float* wk, uint8_t* mask, int32_t* idx, int quant,
-                       cudaStream_t st) {
+// Router, first part: the pass over Q, K (and V) and the column means.
+sla2_status router_head(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
+                        const void* v, int quant, cudaStream_t st) {
   // with V given, its per-channel |V| max (V-hat scales, fp16 scale of the linear state)
   if (v) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
   SLA2_TRY(launch_pool(s, q, k, v, at<float>(d, L.qbar), at<double>(d, L.ksum),
@@ -162,12 +162,55 @@ sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, cons
                        v ? at<unsigned>(d, L.vamax) : nullptr, st));
   SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), at<float>(d, L.kbs),
                            st));
+  return SLA2_OK;
+}
+
+// Router, second part: projections, logits and the hard top-k.
+sla2_status router_tail(const sla2_desc* d, const Shape& s, const Layout& L, const float* wq, const float* wk,
+                        uint8_t* mask, int32_t* idx, cudaStream_t st) {
   SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<float>(d, L.kbs), wq, wk, at<float>(d, L.A),
                        at<float>(d, L.Bk), st));
   float* scores = d->dbg_scores ? d->dbg_scores : at<float>(d, L.scores);
   SLA2_TRY(launch_scores(s, at<float>(d, L.A), at<float>(d, L.Bk), scores, st));
   SLA2_TRY(launch_topk(s, scores, mask, idx, st));
   return SLA2_OK;
+}
+
+sla2_status run_router(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
+                       const void* v, const float* wq, const float* wk, uint8_t* mask, int32_t* idx, int quant,
+                       cudaStream_t st) {
+  sla2_status r = router_head(d, s, L, q, k, v, quant, st);
+  if (r != SLA2_OK) return r;
+  return router_tail(d, s, L, wq, wk, mask, idx, st);
+}
+
+// One auxiliary stream per device, created on the first forward call on that
+// device and kept for the life of the process, on which the router's tail runs
+// while the linear-state pass runs on the caller's stream (the two depend only
+// on the column means). The fork / join events belong to it too; the mutex
+// keeps each call's record / wait pairs together when several host threads
+// enqueue forward calls at once.
+struct AuxStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+AuxStream g_aux[kMaxDevices];
+std::mutex g_aux_mu;
+
+cudaError_t aux_stream(AuxStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  AuxStream& a = g_aux[dev];
+  if (!a.stream) {
+    if ((e = cudaStreamCreateWithFlags(&a.stream, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &a;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -270,9 +313,19 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
 
   uint8_t* mask = at<uint8_t>(desc, L.mask);
   int32_t* idx = at<int32_t>(desc, L.idx);
-  r = run_router(desc, s, L, q, k, v, proj_q, proj_k, mask, idx, quant, st);
+  r = router_head(desc, s, L, q, k, v, quant, st);
   if (r != SLA2_OK) return r;
   SLA2_TRY(mark(1));
+
+  // fork: the router's tail on the auxiliary stream, the linear state on `st`
+  std::lock_guard<std::mutex> aux_lock(g_aux_mu);
+  AuxStream* aux = nullptr;
+  SLA2_TRY(aux_stream(&aux));
+  SLA2_TRY(cudaEventRecord(aux->fork, st));
+  SLA2_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
+  r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, aux->stream);
+  if (r != SLA2_OK) return r;
+  SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
 
   LinearOut o{};
   o.h = at<void>(desc, L.h);
@@ -291,7 +344,15 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, o.vamax, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
                                 at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), st));
+  SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join
   SLA2_TRY(mark(2));
+  // Z_i (needs the top-k and Z_total) on the auxiliary stream, concurrently with the sparse branch
+  if (s.k < s.nk) {
+    SLA2_TRY(cudaEventRecord(aux->fork, st));
+    SLA2_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
+    SLA2_TRY(launch_zsel(s, at<float>(desc, L.Ztot), at<float>(desc, L.z), idx, at<float>(desc, L.Zi), aux->stream));
+    SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
+  }
 
   // sparse branch: tensor maps over the (quantised) operands
   CUtensorMap tq, tk, tv;
@@ -330,7 +391,7 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  if (s.k < s.nk) SLA2_TRY(launch_zsel(s, at<float>(desc, L.Ztot), o.z, idx, at<float>(desc, L.Zi), st));
+  if (s.k < s.nk) SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join (Z_i)
   SLA2_TRY(launch_epilogue(s, ea, st));
   SLA2_TRY(mark(4));
 

@@ -21,9 +21,10 @@
 // MN-major operand layout: the converters overwrite K with phi (fp16) and V
 // with V (fp16) in place, and the MMA reads them as A = V (M = channel) and
 // B = phi (N = feature), both MN-major, K = the 64 tokens.
-// Roles: warps 0-3 convert (quantised copies, phi, z, fp16 operands) and read
-// results back from TMEM; warp 4 lane 0 issues the TMA loads (two stages) and
-// the MMAs.
+// Roles: warps 0-7 convert (quantised copies, phi, z, fp16 operands) and read
+// results back from TMEM (warps w and w + 4 share TMEM lane quadrant w % 4 and
+// split the columns); warp 8 lane 0 issues the TMA loads (two stages) and the
+// MMAs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -34,7 +35,9 @@ namespace sla2 {
 
 namespace {
 
-constexpr int LIN_THREADS = 160;     // 4 converter warps + 1 TMA / MMA warp
+constexpr int LIN_CONV = 256;        // 8 converter warps
+constexpr int LIN_MMA_WARP = 8;      // TMA / MMA warp
+constexpr int LIN_THREADS = LIN_CONV + 32;
 
 template <int D>
 struct LinCfg {
@@ -44,10 +47,10 @@ struct LinCfg {
   static constexpr int OFF_V = KV_TILE;                // V tile (then a zero slab when D = 64: M is 128)
   static constexpr int STAGE = KV_TILE + 2 * SLAB;
   static constexpr int EG = D / 8;                     // feature groups of 8 per token row
-  static constexpr int TG = 128 / EG;                  // token groups
+  static constexpr int TG = LIN_CONV / EG;             // token groups
   static constexpr int TPT = BKB / TG;                 // tokens per converter thread
-  static constexpr int OFF_RED = 2 * STAGE;            // z partials [2][TG][D] + amax [2][4]
-  static constexpr int OFF_BAR = OFF_RED + (2 * TG * D + 8) * 4;
+  static constexpr int OFF_RED = 2 * STAGE;            // z partials [2][TG][D] + amax [2][8]
+  static constexpr int OFF_BAR = OFF_RED + (2 * TG * D + 16) * 4;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;
   static constexpr uint32_t IDESC = make_idesc_mn(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
   static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
@@ -66,8 +69,8 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// named barrier over the 128 converter threads (warps 0-3)
-__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// named barrier over the 256 converter threads (warps 0-7)
+__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __grid_constant__ CUtensorMap tk,
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   extern __shared__ uint8_t lsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
   float* zred_all = reinterpret_cast<float*>(base + C::OFF_RED);     // [2][TG][D]
-  float* ared_all = zred_all + 2 * C::TG * D;                        // [2][4]
+  float* ared_all = zred_all + 2 * C::TG * D;                        // [2][8]
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
   uint64_t* tma_full = bar;          // [2]
   uint64_t* conv_done = bar + 2;
@@ -94,13 +97,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   if (tid == 0) {
     mbar_init(tma_full, 1);
     mbar_init(tma_full + 1, 1);
-    mbar_init(conv_done, 128);
+    mbar_init(conv_done, LIN_CONV);
     mbar_init(mma_done, 1);
     mbar_init(bar + 6, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == LIN_MMA_WARP) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == LIN_MMA_WARP) {
     // ---------------------------------------------------------------- TMA + MMA issuer
     if (lane == 0 && cnt > 0) {
       auto load = [&](int n) {
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- converters (128 threads)
+    // ---------------------------------------------------------------- converters (256 threads)
     constexpr int EG = C::EG, TG = C::TG, TPT = C::TPT;
     const int tg = tid / EG;          // token group: tokens tg*TPT .. +TPT
     const int eg = tid % EG;          // feature / channel group: 8 columns eg*8 ..
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     }
     if (D < 128) {   // channels D..127 of the A operand are a zero slab (the MMA always has M = 128)
       for (int st = 0; st < 2; ++st)
-        for (int t = tid; t < C::SLAB / 16; t += 128)
+        for (int t = tid; t < C::SLAB / 16; t += LIN_CONV)
           *reinterpret_cast<uint4*>(base + st * C::STAGE + C::OFF_V + C::KV_TILE + t * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
     float hs = 1.f;                  // h_mode 2: the head's fp16 operand scale
@@ -182,16 +185,21 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       if (lane == 0) zred_all[warp] = m;
       conv_sync();
-      hs = h_fp16_scale(fmaxf(fmaxf(zred_all[0], zred_all[1]), fmaxf(zred_all[2], zred_all[3])), N);
+      float mx = zred_all[0];
+#pragma unroll
+      for (int w = 1; w < LIN_CONV / 32; ++w) mx = fmaxf(mx, zred_all[w]);
+      hs = h_fp16_scale(mx, N);
       conv_sync();
     }
     float zp = 0.f;                  // this thread's feature (tid < D) partial of Z
-    const uint32_t lane_taddr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int qd = warp & 3, hh = warp >> 2;    // TMEM lane quadrant, column half of the readouts
+    const uint32_t lane_taddr = tmem + ((uint32_t)(qd * 32) << 16);
+    constexpr int RC = D / 2;                   // readout columns per warp
     bool ok = true;
     for (int n = 0; n < cnt; ++n) {
       const int j = j0 + n;
       float* zred = zred_all + (n & 1) * TG * D;
-      float* ared = ared_all + (n & 1) * 4;
+      float* ared = ared_all + (n & 1) * 8;
       ok = mbar_wait(tma_full + (n & 1), (n >> 1) & 1, abort_flag, o.status, o.budget_ns);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       uint8_t* sK = base + (n & 1) * C::STAGE;
@@ -217,7 +225,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
         if (lane == 0) ared[warp] = amax;
         conv_sync();
-        const float a = fmaxf(fmaxf(ared[0], ared[1]), fmaxf(ared[2], ared[3]));
+        const float a = fmaxf(fmaxf(fmaxf(ared[0], ared[1]), fmaxf(ared[2], ared[3])),
+                              fmaxf(fmaxf(ared[4], ared[5]), fmaxf(ared[6], ared[7])));
         const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
 #pragma unroll
         for (int u = 0; u < TPT; ++u) {
@@ -281,25 +290,21 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         for (int c = 0; c < 8; ++c) {
           const size_t orow = ((size_t)bh * nk + j) * D + eg * 8 + c;
           if (o.quant == 1) {
-            uint32_t wq[TPT / 4];
+            uint16_t pr[TPT / 2];
 #pragma unroll
-            for (int u = 0; u < TPT; u += 4) {
-              const uint16_t p0 = cvt_e4m3x2(__fmul_rn(vv[u][c], vinv[c]), __fmul_rn(vv[u + 1][c], vinv[c]));
-              const uint16_t p1 = cvt_e4m3x2(__fmul_rn(vv[u + 2][c], vinv[c]), __fmul_rn(vv[u + 3][c], vinv[c]));
-              wq[u / 4] = (uint32_t)p0 | ((uint32_t)p1 << 16);
-            }
+            for (int u = 0; u < TPT; u += 2)
+              pr[u / 2] = cvt_e4m3x2(__fmul_rn(vv[u][c], vinv[c]), __fmul_rn(vv[u + 1][c], vinv[c]));
             uint8_t* vd = static_cast<uint8_t*>(o.vhatT) + orow * BKB + tg * TPT;
-            if constexpr (TPT == 8)
-              *reinterpret_cast<uint2*>(vd) = make_uint2(wq[0], wq[1]);
+            if constexpr (TPT == 4)
+              *reinterpret_cast<uint32_t*>(vd) = (uint32_t)pr[0] | ((uint32_t)pr[1] << 16);
             else
-              *reinterpret_cast<uint32_t*>(vd) = wq[0];
+              *reinterpret_cast<uint16_t*>(vd) = pr[0];
           } else {
             __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(o.vhatT) + orow * BKB + tg * TPT;
-            if constexpr (TPT == 8)
-              *reinterpret_cast<uint4*>(vd) = make_uint4(cvt_bf16x2(vv[0][c], vv[1][c]), cvt_bf16x2(vv[2][c], vv[3][c]),
-                                                         cvt_bf16x2(vv[4][c], vv[5][c]), cvt_bf16x2(vv[6][c], vv[7][c]));
-            else
+            if constexpr (TPT == 4)
               *reinterpret_cast<uint2*>(vd) = make_uint2(cvt_bf16x2(vv[0][c], vv[1][c]), cvt_bf16x2(vv[2][c], vv[3][c]));
+            else
+              *reinterpret_cast<uint32_t*>(vd) = cvt_bf16x2(vv[0][c], vv[1][c]);
           }
         }
       }
@@ -321,10 +326,11 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       ok = mbar_wait(mma_done, n & 1, abort_flag, o.status, o.budget_ns);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const int c = warp * 32 + lane;
-      if (warp * 32 < D) {
+      const int c = qd * 32 + lane;
+      if (qd * 32 < D) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int c2 = 0; c2 < RC / 32; ++c2) {
+          const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
           uint32_t r[32];
           tmem_ld32(lane_taddr + cc * 32, r);
           tmem_wait_ld();
@@ -359,10 +365,11 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       tc_fence_before();
     }
     // ---- chunk partials (H^T from the accumulating TMEM columns, Z)
-    if (ok && warp * 32 < D) {
-      const int c = warp * 32 + lane;
+    if (ok && qd * 32 < D) {
+      const int c = qd * 32 + lane;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int c2 = 0; c2 < RC / 32; ++c2) {
+        const int cc = hh * (RC / 32) + c2;
         uint32_t r[32];
         tmem_ld32(lane_taddr + C::COL_TOT + cc * 32, r);
         tmem_wait_ld();
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == LIN_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

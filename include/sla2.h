@@ -80,7 +80,9 @@ typedef struct {
   int32_t* dbg_idx;    /* selected block indices, ascending, [B][H][N/128][k]   */
   /* Optional timing hooks: NULL, or an array of SLA2_STAGE_EVENTS cudaEvent_t
      that sla2_forward records on `stream` at the stage boundaries
-     [start, router done, linear state done, sparse branch done, end].       */
+     [start, pass over Q/K/V and column means done, linear state and router
+     tail (projections, logits, top-k; run concurrently) done, sparse branch
+     done, end].                                                             */
   void* const* stage_events;
 } sla2_desc;
 
@@ -157,6 +159,13 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
 /* The whole forward pass (steps 1-4): out = alpha O_s + (1 - alpha) O_l.
  *   out : bf16 or fp32 (desc->out_dtype) [B][H][N][d]
  * All intermediates live in desc->workspace; optional debug exports in desc.
+ * The router's projections, logits and top-k run on a library-owned
+ * non-blocking stream, forked from and joined back into `stream` with events,
+ * concurrently with the linear-state pass. That stream and its two events are
+ * created by the first call on each device and kept until the process exits;
+ * make that first call outside any stream capture. Later calls can be captured
+ * (the fork and join become graph edges). Calls from several host threads are
+ * serialised while they enqueue.
  * Arithmetic: router in fp32; sparse branch INT8 Q K^T (int32 accumulate) and
  * e4m3 P V (fp32 accumulate) with quantize = 1, bf16 operands with quantize = 0;
  * linear branch on fp16 tensor-core operands with fp32 accumulation, h_j and
