@@ -8,7 +8,7 @@
 //   K_s   = fp32(K) - fp32(c)                      (K smoothing, detail §7 note 1)
 //   K-hat = INT8 of K_s over the 64 x d block, s_k = amax / 127
 //   V-hat^T = e4m3(V * 448 / amax_channel), channel-major [d][64]
-//   phi   = softmax of each K_s row over the d features (fp32, accurate expf)
+//   phi   = softmax of each K_s row over the d features (fp32, ex2.approx)
 //   z_j   = sum over the block's tokens of phi                   (fp32)
 //   h_j^T = V_j^T phi_j  on the tensor core: tcgen05 kind::f16 with fp16
 //           operands (V exactly, phi rounded once), fp32 accumulation in TMEM;
@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   uint64_t* mma_done = bar + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
   int* abort_flag = reinterpret_cast<int*>(bar + 5);        // bar + 6: drain barrier
+  uint64_t* rd_done = bar + 7;       // the per-block accumulator has been read
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y, chunk = blockIdx.x, G = gridDim.x;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     mbar_init(conv_done, LIN_CONV);
     mbar_init(mma_done, 1);
     mbar_init(bar + 6, 1);
+    mbar_init(rd_done, LIN_CONV);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -130,6 +132,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       bool ok = true;
       for (int n = 0; n < cnt; ++n) {
         if (!mbar_wait(conv_done, n & 1, abort_flag, o.status, o.budget_ns)) { ok = false; break; }
+        // the per-block accumulator is free once block n - 1 has been read out of it
+        if (n >= 1 && !mbar_wait(rd_done, (n - 1) & 1, abort_flag, o.status, o.budget_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t stg = smem_u32(base + (n & 1) * C::STAGE);
 #pragma unroll
@@ -195,6 +199,58 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     const int qd = warp & 3, hh = warp >> 2;    // TMEM lane quadrant, column half of the readouts
     const uint32_t lane_taddr = tmem + ((uint32_t)(qd * 32) << 16);
     constexpr int RC = D / 2;                   // readout columns per warp
+    // h_j^T of block nn: TMEM lane c (one channel per thread) -> registers, the
+    // accumulator released to the next block's MMA, then fp16 / bf16 / fp32 -> global
+    auto readout = [&](int nn) -> bool {
+      const int j = j0 + nn;
+      bool rok = mbar_wait(mma_done, nn & 1, abort_flag, o.status, o.budget_ns);
+      if (!__all_sync(0xffffffffu, rok)) return false;
+      tc_fence_after();
+      const int c = qd * 32 + lane;
+      uint32_t rr[RC / 32][32];
+      if (qd * 32 < D) {
+#pragma unroll
+        for (int c2 = 0; c2 < RC / 32; ++c2) tmem_ld32(lane_taddr + (hh * (RC / 32) + c2) * 32, rr[c2]);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(rd_done);
+      if (qd * 32 < D) {
+#pragma unroll
+        for (int c2 = 0; c2 < RC / 32; ++c2) {
+          const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
+          const uint32_t (&r)[32] = rr[c2];
+          if (o.h_mode == 2) {
+            uint8_t* tile = static_cast<uint8_t*>(o.h) + ((size_t)bh * nk + j) * (size_t)(D * D * 2);
+            const float ns = -hs;
+#pragma unroll
+            for (int q = 0; q < 32; q += 8)
+              *reinterpret_cast<uint4*>(tile + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
+                  h2_bits(ns * __uint_as_float(r[q]), ns * __uint_as_float(r[q + 1])),
+                  h2_bits(ns * __uint_as_float(r[q + 2]), ns * __uint_as_float(r[q + 3])),
+                  h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
+                  h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
+          } else if (o.h_mode == 1) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+#pragma unroll
+            for (int q = 0; q < 32; q += 8)
+              *reinterpret_cast<uint4*>(dst + q) = make_uint4(
+                  cvt_bf16x2(__uint_as_float(r[q]), __uint_as_float(r[q + 1])),
+                  cvt_bf16x2(__uint_as_float(r[q + 2]), __uint_as_float(r[q + 3])),
+                  cvt_bf16x2(__uint_as_float(r[q + 4]), __uint_as_float(r[q + 5])),
+                  cvt_bf16x2(__uint_as_float(r[q + 6]), __uint_as_float(r[q + 7])));
+          } else {
+            float* dst = static_cast<float*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+#pragma unroll
+            for (int q = 0; q < 32; q += 4)
+              *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                                                __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
+          }
+        }
+      }
+      return true;
+    };
+
     bool ok = true;
     for (int n = 0; n < cnt; ++n) {
       const int j = j0 + n;
@@ -252,15 +308,17 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         for (int c = 1; c < 8; ++c) m = fmaxf(m, x[u][c]);
 #pragma unroll
         for (int off = EG / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        // exp(x - m) as 2^(x log2 e - m log2 e); phi is rounded to fp16 for the MMA
+        const float mb = m * 1.4426950408889634f;
         float sum = 0.f;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          x[u][c] = expf(x[u][c] - m);
+          x[u][c] = ex2_approx(fmaf(x[u][c], 1.4426950408889634f, -mb));
           sum += x[u][c];
         }
 #pragma unroll
         for (int off = EG / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        const float inv = 1.f / sum;
+        const float inv = __frcp_rn(sum);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           x[u][c] *= inv;          // phi
@@ -322,48 +380,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         o.z[((size_t)bh * nk + j) * D + tid] = z;
         zp += z;
       }
-      // ---- h_j^T: TMEM lane c (one channel per thread) -> global
-      ok = mbar_wait(mma_done, n & 1, abort_flag, o.status, o.budget_ns);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const int c = qd * 32 + lane;
-      if (qd * 32 < D) {
-#pragma unroll
-        for (int c2 = 0; c2 < RC / 32; ++c2) {
-          const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
-          uint32_t r[32];
-          tmem_ld32(lane_taddr + cc * 32, r);
-          tmem_wait_ld();
-          if (o.h_mode == 2) {
-            uint8_t* tile = static_cast<uint8_t*>(o.h) + ((size_t)bh * nk + j) * (size_t)(D * D * 2);
-            const float ns = -hs;
-#pragma unroll
-            for (int q = 0; q < 32; q += 8)
-              *reinterpret_cast<uint4*>(tile + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
-                  h2_bits(ns * __uint_as_float(r[q]), ns * __uint_as_float(r[q + 1])),
-                  h2_bits(ns * __uint_as_float(r[q + 2]), ns * __uint_as_float(r[q + 3])),
-                  h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
-                  h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
-          } else if (o.h_mode == 1) {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
-#pragma unroll
-            for (int q = 0; q < 32; q += 8)
-              *reinterpret_cast<uint4*>(dst + q) = make_uint4(
-                  cvt_bf16x2(__uint_as_float(r[q]), __uint_as_float(r[q + 1])),
-                  cvt_bf16x2(__uint_as_float(r[q + 2]), __uint_as_float(r[q + 3])),
-                  cvt_bf16x2(__uint_as_float(r[q + 4]), __uint_as_float(r[q + 5])),
-                  cvt_bf16x2(__uint_as_float(r[q + 6]), __uint_as_float(r[q + 7])));
-          } else {
-            float* dst = static_cast<float*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
-#pragma unroll
-            for (int q = 0; q < 32; q += 4)
-              *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
-                                                                __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
-          }
-        }
+      // ---- h_j^T of the previous block (its MMA ran while this block was converted)
+      if (n >= 1 && !readout(n - 1)) {
+        ok = false;
+        break;
       }
-      tc_fence_before();
     }
+    if (ok && cnt >= 1) ok = readout(cnt - 1);
     // ---- chunk partials (H^T from the accumulating TMEM columns, Z)
     if (ok && qd * 32 < D) {
       const int c = qd * 32 + lane;
