@@ -438,8 +438,10 @@ __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const floa
     if (blockIdx.x == 0 && threadIdx.x == 0 && hscale) hscale[bh] = hs;
   }
   if (e < DD) {
+    // fixed summation order; the loads are independent, so batches of them are issued together
     float s = 0.f;
-    for (int g = 0; g < G; ++g) s += hpart[((size_t)bh * G + g) * DD + e];
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) s += __ldg(hpart + ((size_t)bh * G + g) * DD + e);
     Htot[(size_t)bh * DD + e] = s;
     if (vamax && htile) {
       const int row = e / D, col = e % D;
@@ -449,7 +451,8 @@ __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const floa
   }
   if (blockIdx.x == 0 && threadIdx.x < D) {
     float s = 0.f;
-    for (int g = 0; g < G; ++g) s += zpart[((size_t)bh * G + g) * D + threadIdx.x];
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) s += __ldg(zpart + ((size_t)bh * G + g) * D + threadIdx.x);
     Ztot[(size_t)bh * D + threadIdx.x] = s;
   }
 }

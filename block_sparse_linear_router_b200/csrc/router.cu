@@ -62,6 +62,12 @@ __global__ void __launch_bounds__(256, 2) pool_kernel(const __nv_bfloat16* __res
   const int cg = tid % TPR, rg = tid / TPR;
   const size_t base = ((size_t)bh * N + (size_t)i * BQ) * D + cg * 8;
 
+  // V is read last: start bringing its rows into L2 now (one prefetch per 128-byte line)
+  if (vamax && (cg & 7) == 0) {
+#pragma unroll
+    for (int p = 0; p < NP; ++p)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(v + base + (size_t)(p * RPP + rg) * D)));
+  }
   uint4 wq[NP], wk[NP];
 #pragma unroll
   for (int p = 0; p < NP; ++p) wq[p] = __ldg(reinterpret_cast<const uint4*>(q + base + (size_t)(p * RPP + rg) * D));
