@@ -261,6 +261,30 @@ sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k, con
   return SLA2_OK;
 }
 
+sla2_status sla2_router_soft(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
+                             const float* proj_k, float topk_frac, float tau, float* soft_out, float* lambda_out,
+                             void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !proj_q || !proj_k || !soft_out) return SLA2_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !(tau < INFINITY)) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  r = router_head(desc, s, L, q, k, nullptr, 0, st);
+  if (r != SLA2_OK) return r;
+  SLA2_TRY(launch_proj(s, desc->H, at<float>(desc, L.qbar), at<float>(desc, L.kbs), proj_q, proj_k,
+                       at<float>(desc, L.A), at<float>(desc, L.Bk), st));
+  float* scores = desc->dbg_scores ? desc->dbg_scores : at<float>(desc, L.scores);
+  SLA2_TRY(launch_scores(s, at<float>(desc, L.A), at<float>(desc, L.Bk), scores, st));
+  SLA2_TRY(launch_soft_topk(s, scores, tau, soft_out, lambda_out, st));
+  return SLA2_OK;
+}
+
 sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v, const float* colmean,
                               float* h_out, float* z_out, float* Htot_out, float* Ztot_out, void* stream) {
   Shape s;

@@ -37,6 +37,9 @@ cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float
 // hard top-k per logit row (ties -> lower index), mask and ascending index list
 cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st);
 int scores_topk_max_nk();
+// SoftTop-k relaxation of each logit row: sigmoid(P_c / tau + lambda), row sums k
+cudaError_t launch_soft_topk(const Shape& s, const float* scores, float tau, float* soft, float* lam,
+                             cudaStream_t st);
 
 // ---- linear state (linear.cu) ---------------------------------------------
 // Per key block: h_j, z_j (fp32) and per-chunk partial sums; optionally K-hat /

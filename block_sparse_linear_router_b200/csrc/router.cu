@@ -321,7 +321,70 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
   }
 }
 
+// SoftTop-k of one logit row per warp (SLA2 detail page §4, Eq. 17): P_c = row
+// softmax of the logits, m_j = sigmoid(P_c[j] / tau + lambda) with lambda found
+// by bisection on [logit(k / nk) - 1 / tau, logit(k / nk)] so that the row sums
+// to k. x = P_c / tau is kept in shared memory for the bisection passes.
+constexpr int SOFT_ITERS = 48;        // halvings of a bracket 1 / tau wide: below fp32 resolution
+
+__global__ void __launch_bounds__(TOPK_WARPS * 32) soft_topk_kernel(const float* __restrict__ scores, int rows,
+                                                                    int nk, int k, float tau,
+                                                                    float* __restrict__ soft,
+                                                                    float* __restrict__ lam_out) {
+  extern __shared__ float xs_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * TOPK_WARPS + warp;
+  if (row >= rows) return;
+  float* xs = xs_all + (size_t)warp * nk;
+  const float* srow = scores + (size_t)row * nk;
+  float* out = soft + (size_t)row * nk;
+  if (k >= nk) {                      // every block kept: the relaxation is identically 1
+    for (int j = lane; j < nk; j += 32) out[j] = 1.f;
+    if (lam_out && lane == 0) lam_out[row] = INFINITY;
+    return;
+  }
+  float m = -INFINITY;
+  for (int j = lane; j < nk; j += 32) m = fmaxf(m, srow[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+  for (int j = lane; j < nk; j += 32) {
+    const float e = expf(srow[j] - m);
+    xs[j] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float scale = 1.f / (sum * tau);          // x = P_c / tau
+  for (int j = lane; j < nk; j += 32) xs[j] *= scale;
+  __syncwarp();
+  const float base = logf((float)k / (float)(nk - k));
+  float lo = base - 1.f / tau, hi = base;
+  for (int itn = 0; itn < SOFT_ITERS; ++itn) {
+    const float mid = 0.5f * (lo + hi);
+    float f = 0.f;
+    for (int j = lane; j < nk; j += 32) f += 1.f / (1.f + expf(-(xs[j] + mid)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+    if (f < (float)k) lo = mid;
+    else hi = mid;
+  }
+  const float lam = 0.5f * (lo + hi);
+  for (int j = lane; j < nk; j += 32) out[j] = 1.f / (1.f + expf(-(xs[j] + lam)));
+  if (lam_out && lane == 0) lam_out[row] = lam;
+}
+
 }  // namespace
+
+cudaError_t launch_soft_topk(const Shape& s, const float* scores, float tau, float* soft, float* lam,
+                             cudaStream_t st) {
+  const int rows = s.BH * s.nq;
+  const size_t smem = (size_t)TOPK_WARPS * s.nk * sizeof(float);
+  cudaFuncSetAttribute(soft_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  soft_topk_kernel<<<(rows + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(scores, rows, s.nk, s.k, tau,
+                                                                                         soft, lam);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void* v, float* qbar, double* ksum,
                         int8_t* qhat, float* sq, unsigned* vamax, cudaStream_t st) {

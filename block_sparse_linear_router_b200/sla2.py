@@ -49,6 +49,8 @@ SIGNATURES = {
     "sla2_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Desc), ctypes.c_float]),
     "sla2_router": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 4 + [ctypes.c_float]
                     + [ctypes.c_void_p] * 4),
+    "sla2_router_soft": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 4
+                         + [ctypes.c_float, ctypes.c_float] + [ctypes.c_void_p] * 3),
     "sla2_linear_state": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 8),
     "sla2_forward": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 6 + [ctypes.c_float]
                      + [ctypes.c_void_p] * 2),
@@ -142,6 +144,32 @@ def router(q, k, proj_q, proj_k, frac, workspace: Optional[Workspace] = None, sc
     if r != 0:
         raise Sla2Error(r, "sla2_router")
     out = {"mask": mask, "idx": idx, "colmean": cm}
+    if sc is not None:
+        out["scores"] = sc
+    return out
+
+
+def router_soft(q, k, proj_q, proj_k, frac, tau=0.1, workspace: Optional[Workspace] = None, scores=False,
+                stream=None):
+    """SoftTop-k mask sigmoid(P_c / tau + lambda) (fp32 [B,H,nq,nk], rows summing to k) and lambda
+    (fp32 [B,H,nq]); optionally the fp32 logits."""
+    lib = load_library()
+    _check_qkv(q, k, proj_q, proj_k)
+    B, H, N, d = q.shape
+    nq, nk = N // 128, N // 64
+    ws = workspace or Workspace.for_shape(B, H, N, d, frac, 0, q.device)
+    desc = make_desc(B, H, N, d, 0)
+    desc.workspace, desc.workspace_bytes = ws.buf.data_ptr(), ws.buf.numel()
+    soft = torch.empty(B, H, nq, nk, dtype=torch.float32, device=q.device)
+    lam = torch.empty(B, H, nq, dtype=torch.float32, device=q.device)
+    sc = torch.empty(B, H, nq, nk, dtype=torch.float32, device=q.device) if scores else None
+    if sc is not None:
+        desc.dbg_scores = sc.data_ptr()
+    r = lib.sla2_router_soft(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(proj_q), _ptr(proj_k), frac, tau,
+                             _ptr(soft), _ptr(lam), _stream(stream))
+    if r != 0:
+        raise Sla2Error(r, "sla2_router_soft")
+    out = {"soft": soft, "lambda": lam}
     if sc is not None:
         out["scores"] = sc
     return out

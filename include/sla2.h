@@ -113,6 +113,19 @@ sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k,
                         uint8_t* mask_out, int32_t* idx_out, float* colmean_out,
                         void* stream);
 
+/* SoftTop-k relaxation of the router's mask (detail page §4, Eq. 17; the
+ * training-time mask of summary step 1):
+ *   soft_out[b][h][i][j] = sigmoid(P_c[i][j] / tau + lambda_i),  fp32 [B][H][N/128][N/64]
+ *   lambda_out[b][h][i]  = lambda_i (fp32 [B][H][N/128]) or NULL
+ * P_c is the row softmax of the router logits of sla2_router; lambda_i is found
+ * by bisection so that every row sums to k, the number of blocks the hard
+ * Top-k keeps (k = nk gives all ones and lambda = +inf). tau must be positive
+ * and finite (the pages use 0.1); otherwise SLA2_ERR_INVALID_ARG. Uses
+ * desc->workspace; desc->dbg_scores receives the logits when non-NULL. */
+sla2_status sla2_router_soft(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
+                             const float* proj_k, float topk_frac, float tau, float* soft_out,
+                             float* lambda_out, void* stream);
+
 /* The router of sla2_router, for callers that cannot allocate device memory
  * (no counterpart on the SLA2 pages; an addition of this library). Some
  * callers may not call cudaMalloc at all: a plugin inside a host framework

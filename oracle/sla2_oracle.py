@@ -33,7 +33,9 @@ the design notes):
     unquantised P; the linear branch is not quantised;
   * online-softmax schedule (mode "qa"): one running-max update per selected
     key block, key blocks in ascending index order;
-  * k = nk: the linear branch is defined as 0 (no unselected blocks).
+  * k = nk: the linear branch is defined as 0 (no unselected blocks);
+  * SoftTop-k ([D] §4 Eq. 17): "each row sums to k%" is read as the row
+    summing to k, the count of blocks the hard Top-k keeps; lambda by bisection.
 
 Modes of ``forward``:
   "qa" quantised, online softmax in the tile order above (the contract);
@@ -111,6 +113,54 @@ def topk_mask(s: np.ndarray, k: int):
         mask[i, sel] = 1
         idx[i] = sel
     return mask, idx
+
+
+def soft_topk(pc_row: np.ndarray, k: int, tau: float, iters: int = 200):
+    """SoftTop-k of one row of P_c ([D] §4 Eq. 17; [S] step 1, the training-time
+    mask): m_j = sigmoid(P_c[j] / tau + lambda), with the row offset lambda
+    found by bisection so that the row sums to k (the number of blocks the hard
+    Top-k keeps). The row sum is strictly increasing in lambda; because
+    P_c / tau lies in [0, 1 / tau], the root lies in
+    [logit(k / nk) - 1 / tau, logit(k / nk)]. Returns (mask row, lambda); for
+    k = nk every entry is 1 and lambda is +inf."""
+    x = np.asarray(pc_row, dtype=np.float64) / tau
+    nk = x.shape[0]
+    if k >= nk:
+        return np.ones(nk), math.inf
+    target = float(k)
+    base = math.log(k / (nk - k))
+    lo, hi = base - 1.0 / tau, base
+
+    def sig(t):
+        with np.errstate(over="ignore"):      # exp overflow -> sigmoid 0, as intended
+            return 1.0 / (1.0 + np.exp(-t))
+
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        if float(np.sum(sig(x + mid))) < target:
+            lo = mid
+        else:
+            hi = mid
+    lam = 0.5 * (lo + hi)
+    return sig(x + lam), lam
+
+
+def router_soft(q, k, proj_q, proj_k, frac, tau):
+    """SoftTop-k masks and offsets for [B, H, N, d] inputs: float64
+    [B, H, nq, nk] and [B, H, nq]."""
+    q, k = (np.asarray(t.float() if hasattr(t, "float") else t, dtype=np.float64) for t in (q, k))
+    B, H, N, d = q.shape
+    nq, nk = N // BQ, N // BK
+    kk = topk_count(nk, frac)
+    soft = np.zeros((B, H, nq, nk))
+    lam = np.zeros((B, H, nq))
+    for b in range(B):
+        for hh in range(H):
+            s = router_scores(q[b, hh], k[b, hh], np.asarray(proj_q[hh], np.float64), np.asarray(proj_k[hh], np.float64))
+            pc = compressed_probs(s)
+            for i in range(nq):
+                soft[b, hh, i], lam[b, hh, i] = soft_topk(pc[i], kk, tau)
+    return soft, lam
 
 
 # --------------------------------------------------------------------------

@@ -110,6 +110,17 @@ def test_router_and_linear_state_argument_errors(lib):
     assert lib.sla2_linear_state(ctypes.byref(_desc()), v, v, v, v, v, v, v, None) == 3
 
 
+def test_router_soft_argument_errors(lib):
+    keep, p = _fake()
+    v = ctypes.c_void_p(p)
+    for tau in (0.0, -0.1, float("inf"), float("nan")):
+        assert lib.sla2_router_soft(ctypes.byref(_desc()), v, v, v, v, 0.1, tau, v, None, None) == 1
+    assert lib.sla2_router_soft(ctypes.byref(_desc()), v, v, v, v, 0.0, 0.1, v, None, None) == 1     # frac
+    assert lib.sla2_router_soft(ctypes.byref(_desc()), v, v, v, v, 0.1, 0.1, None, None, None) == 1  # no output
+    assert lib.sla2_router_soft(ctypes.byref(_desc(d=96)), v, v, v, v, 0.1, 0.1, v, None, None) == 2
+    assert lib.sla2_router_soft(ctypes.byref(_desc()), v, v, v, v, 0.1, 0.1, v, None, None) == 3      # workspace
+
+
 def test_selftest_rejects_bad_arguments(lib):
     lib.sla2_selftest_timeout.restype = ctypes.c_int
     lib.sla2_selftest_timeout.argtypes = [ctypes.c_void_p, ctypes.c_ulonglong, ctypes.c_void_p]

@@ -175,6 +175,34 @@ def test_router_entry_point(sla2):
     np.testing.assert_array_equal(r["colmean"].cpu().numpy(), cm.astype(np.float32))
 
 
+def test_router_identity_projection_is_heuristic_router(sla2):
+    # proj = I: the learnable router reduces to the pooled-attention Top-k of SLA (detail page §2)
+    inp = make_custom(1, 3, 2048, 64, 0.1, seed=31)
+    eye = torch.eye(64).expand(3, 64, 64).contiguous()
+    dev = to_dev(inp)
+    r = sla2.router(dev["q"], dev["k"], eye.cuda(), eye.cuda(), 0.1, scores=True)
+    mask, idx, scores = O.router(inp.q, inp.k, eye, eye, 0.1)
+    check_mask_rows(r["mask"].cpu().numpy(), mask, scores, O.topk_count(32, 0.1))
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 2048, 64, 0.1, 0.1), (1, 2, 8192, 128, 0.03, 0.1), (2, 1, 1024, 64, 0.3, 0.5)])
+def test_router_soft_matches_oracle(sla2, shape):
+    B, H, N, d, frac, tau = shape
+    inp = make_custom(B, H, N, d, frac, seed=32)
+    dev = to_dev(inp)
+    r = sla2.router_soft(dev["q"], dev["k"], dev["proj_q"], dev["proj_k"], frac, tau=tau)
+    soft, lam = O.router_soft(inp.q, inp.k, inp.proj_q, inp.proj_k, frac, tau)
+    got = r["soft"].cpu().numpy()
+    kk = O.topk_count(N // 64, frac)
+    e_soft = float(np.max(np.abs(got - soft)))
+    e_lam = float(np.max(np.abs(r["lambda"].cpu().numpy() - lam)))
+    e_sum = float(np.max(np.abs(got.sum(-1) - kk)))
+    print(f"router_soft {shape}: max|soft| {e_soft:.2e} max|lambda| {e_lam:.2e} max|row sum - k| {e_sum:.2e}")
+    assert e_soft < 2e-5          # fp32 logits, softmax and sigmoids against fp64
+    assert e_lam < 1e-4
+    assert e_sum < 1e-3
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_linear_state_entry_point(sla2, d):
     inp = make_custom(1, 2, 1024, d, 0.1, seed=29)

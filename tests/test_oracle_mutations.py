@@ -95,3 +95,12 @@ def test_missing_mix_complement_is_caught(monkeypatch):
         return r
     monkeypatch.setattr(O, "head_forward", wrong)
     assert _fails(pins.test_constant_keys_closed_form)
+
+
+def test_soft_topk_temperature_multiplied_is_caught(monkeypatch):
+    orig = O.soft_topk
+
+    def wrong(pc_row, k, tau, iters=200):
+        return orig(np.asarray(pc_row) * tau * tau, k, tau, iters)   # P_c * tau instead of P_c / tau
+    monkeypatch.setattr(O, "soft_topk", wrong)
+    assert _fails(pins.test_soft_topk_small_tau_is_hard_topk)

@@ -325,3 +325,51 @@ def test_quantised_k_is_smoothed():
     for j in range(8):
         deq = kh[j * 64:(j + 1) * 64].astype(np.float64) * float(sk[j])
         assert np.max(np.abs(deq - Ks[j * 64:(j + 1) * 64])) <= 0.5 * float(sk[j]) * 1.001 + 1e-6
+
+
+# --------------------------------------------------------------------------
+# SoftTop-k (detail page §4, Eq. 17): sigmoid(P_c / tau + lambda_i), lambda_i
+# by bisection so that each row sums to k
+# --------------------------------------------------------------------------
+def test_soft_topk_rows_sum_to_k_and_lambda_in_bracket():
+    rng = np.random.default_rng(11)
+    for nk, frac, tau in ((32, 0.1, 0.1), (512, 0.03, 0.1), (256, 0.5, 0.05), (40, 0.25, 1.0)):
+        k = O.topk_count(nk, frac)
+        pc = rng.random(nk) ** 3
+        pc /= pc.sum()
+        m, lam = O.soft_topk(pc, k, tau)
+        assert abs(m.sum() - k) < 1e-9
+        assert np.all((m > 0) & (m < 1))
+        base = math.log(k / (nk - k))
+        assert base - 1.0 / tau - 1e-12 <= lam <= base + 1e-12
+
+
+def test_soft_topk_constant_row_closed_form():
+    # every P_c equal: sigmoid(c / tau + lambda) = k / nk for every entry
+    for nk, k, tau in ((32, 3, 0.1), (512, 15, 0.1), (64, 40, 0.5)):
+        m, lam = O.soft_topk(np.full(nk, 1.0 / nk), k, tau)
+        np.testing.assert_allclose(m, k / nk, rtol=0, atol=1e-12)
+        assert abs(lam - (math.log(k / (nk - k)) - 1.0 / (nk * tau))) < 1e-9
+
+
+def test_soft_topk_small_tau_is_hard_topk():
+    # well separated P_c and a tiny temperature: the relaxation reaches the hard mask
+    rng = np.random.default_rng(12)
+    nk, k = 64, 7
+    pc = rng.permutation(np.arange(1, nk + 1, dtype=np.float64))
+    pc /= pc.sum()                     # neighbouring values differ by 1 / sum = 4.8e-4
+    m, _ = O.soft_topk(pc, k, 2e-5)
+    hard = np.zeros(nk)
+    hard[np.argsort(-pc)[:k]] = 1.0
+    assert np.max(np.abs(m - hard)) < 1e-3
+
+
+def test_soft_topk_preserves_order_and_full_selection():
+    rng = np.random.default_rng(13)
+    pc = rng.random(100)
+    pc /= pc.sum()
+    m, _ = O.soft_topk(pc, 10, 0.1)
+    order = np.argsort(pc)
+    assert np.all(np.diff(m[order]) >= 0)
+    m_all, lam = O.soft_topk(pc, 100, 0.1)
+    assert np.all(m_all == 1.0) and lam == math.inf
