@@ -155,6 +155,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(x, dist, device):
+    """The slowest rank's value: a MAX all-reduce that every rank takes part in (the
+    job's time is the time of its slowest rank)."""
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ops_per_step, ms_per_step, world_size):
+    """Whole-job throughput in TOPS: every rank runs one replica of the workload per
+    step, and the step time is the slowest rank's."""
+    return ops_per_step / (ms_per_step * 1e-3) / 1e12 * world_size
+
+
 def dist_setup():
     import torch
     import torch.distributed as dist
@@ -305,12 +320,10 @@ def main():
             stage_ms[s] += row[s].elapsed_time(row[s + 1]) / K
     ms_step = ms_total / K
     if ws > 1:
-        tt = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+        ms_step = max_over_ranks(ms_step, dist, dev)
 
     wm = work_model(w, k)
-    eff_tops = wm["effective_ops"] / (ms_step * 1e-3) / 1e12 * ws
+    eff_tops = job_throughput(wm["effective_ops"], ms_step, ws)
 
     # ---- end to end through the public API: pinned host inputs -> device -> forward -> host output
     e2e = None
@@ -343,10 +356,8 @@ def main():
         torch.cuda.synchronize(dev)
         ms_e2e = f0.elapsed_time(f1) / ke
         if ws > 1:
-            tt = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms_e2e = float(tt.item())
-        e2e = {"value": wm["effective_ops"] / (ms_e2e * 1e-3) / 1e12 * ws, "unit": "TOPS",
+            ms_e2e = max_over_ranks(ms_e2e, dist, dev)
+        e2e = {"value": job_throughput(wm["effective_ops"], ms_e2e, ws), "unit": "TOPS",
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
