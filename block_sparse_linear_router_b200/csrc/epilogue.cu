@@ -90,12 +90,13 @@ __device__ __forceinline__ uint32_t h2(float lo, float hi) {
 }
 
 // Read-only 16-byte load kept where it is written (its latency overlaps the
-// work in between instead of being moved down to the first use).
-__device__ __forceinline__ uint4 ldg_v4_early(const uint4* p) {
+// work in between instead of being moved down to the first use), with an L2
+// cache policy.
+__device__ __forceinline__ uint4 ldg_v4_early(const uint4* p, uint64_t pol) {
   uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(reinterpret_cast<uint64_t>(p)));
+               : "l"(reinterpret_cast<uint64_t>(p)), "l"(pol));
   return r;
 }
 
@@ -119,9 +120,10 @@ __device__ __forceinline__ bool compute_sync_any(bool failed) {
   return r != 0;
 }
 
-// O = alpha O_s + (1 - alpha) O_l for 32 consecutive columns of one row.
+// O = alpha O_s + (1 - alpha) O_l for 32 consecutive columns of one row
+// (stored with the streaming L2 policy `pol`).
 __device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, float alpha, const float4* osv,
-                                          const float* ol) {
+                                          const float* ol, uint64_t pol) {
   float o[32];
 #pragma unroll
   for (int c = 0; c < 32; c += 4) {
@@ -139,13 +141,18 @@ __device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, flo
   if (a.out_f32) {
 #pragma unroll
     for (int c = 0; c < 32; c += 4)
-      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + off + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+      stg_u4_policy(static_cast<float*>(a.out) + off + c,
+                    make_uint4(__float_as_uint(o[c]), __float_as_uint(o[c + 1]), __float_as_uint(o[c + 2]),
+                               __float_as_uint(o[c + 3])),
+                    pol);
   } else {
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + off;
 #pragma unroll
     for (int c = 0; c < 32; c += 8)
-      *reinterpret_cast<uint4*>(dst + c) = make_uint4(cvt_bf16x2(o[c], o[c + 1]), cvt_bf16x2(o[c + 2], o[c + 3]),
-                                                      cvt_bf16x2(o[c + 4], o[c + 5]), cvt_bf16x2(o[c + 6], o[c + 7]));
+      stg_u4_policy(dst + c,
+                    make_uint4(cvt_bf16x2(o[c], o[c + 1]), cvt_bf16x2(o[c + 2], o[c + 3]), cvt_bf16x2(o[c + 4], o[c + 5]),
+                               cvt_bf16x2(o[c + 6], o[c + 7])),
+                    pol);
   }
 }
 
@@ -206,6 +213,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
     const int pr = warp == EPI_PRODUCER_WARP0 ? 0 : 1;   // this producer's tiles: t = pr, pr + 2, ...
     if (lane == 0 && has_linear) {
       const size_t tile_elems = (size_t)D * D;
+      const uint64_t keep = l2_policy_evict_last();   // a tile is re-read by ~k query blocks of the head
       int st = 0, ng = 0, it = 0, nz = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -235,7 +243,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
             const int n = n0 + t;
             const uint16_t* src = n == 0 ? a.htile + (size_t)bh * tile_elems
                                          : a.hT + ((size_t)bh * s.nk + __ldg(sel + n - 1)) * tile_elems;
-            bulk_load(dst + t * C::TILE, src, C::TILE, full + st);
+            bulk_load_hint(dst + t * C::TILE, src, C::TILE, full + st, keep);
           }
           ++ng;
           if (++st == C::NS) {
@@ -298,6 +306,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
     const int qd = warp & 3, fh = warp >> 2;     // TMEM lane quadrant, feature / column half
     const int r = qd * 32 + lane;                // query row of the block = TMEM lane
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    const uint64_t stream_pol = l2_policy_evict_first();   // Q, O_s and out are touched once here
     auto row_of = [&](int w) { return (size_t)(w / s.nq) * s.N + (size_t)(w % s.nq) * BQ + r; };
 
     if (!has_linear) {
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
           const float4* osr = reinterpret_cast<const float4*>(a.os + row * D + fh * HC + cc * 32);
 #pragma unroll
           for (int c = 0; c < 8; ++c) osv[c] = __ldg(osr + c);
-          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, zero);
+          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, zero, stream_pol);
         }
       }
     } else {
@@ -329,7 +338,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         const float* osr = a.os + row * D + fh * HC;
         float4 osv[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr) + c);
+        for (int c = 0; c < 8; ++c) osv[c] = ldg_f4_policy(reinterpret_cast<const float4*>(osr) + c, stream_pol);
         bool ok = mbar_wait(dfull, itp & 1, abort_flag, a.status, a.budget_ns);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
@@ -358,9 +367,9 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         for (int cc = 0; cc < HC / 32; ++cc) {
           if (cc > 0) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) osv[c] = __ldg(reinterpret_cast<const float4*>(osr + cc * 32) + c);
+            for (int c = 0; c < 8; ++c) osv[c] = ldg_f4_policy(reinterpret_cast<const float4*>(osr + cc * 32) + c, stream_pol);
           }
-          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, ol + cc * 32);
+          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, ol + cc * 32, stream_pol);
         }
         return true;
       };
@@ -369,7 +378,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
       auto load_q = [&](int w) {               // issued here, consumed one item later
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row_of(w) * D + fh * HC);
 #pragma unroll
-        for (int i = 0; i < HC / 8; ++i) qv[i] = ldg_v4_early(src + i);
+        for (int i = 0; i < HC / 8; ++i) qv[i] = ldg_v4_early(src + i, stream_pol);
       };
       load_q(blockIdx.x);
       int it = 0, wprev = -1;

@@ -321,6 +321,52 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
   }
 }
 
+// The same hard Top-k with the row held in registers (NPL keys per lane, row
+// lengths up to 32 NPL): one compare per key and one warp reduction per bit.
+template <int NPL>
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_reg_kernel(const float* __restrict__ scores, int rows, int nk,
+                                                                   int k, uint8_t* __restrict__ mask,
+                                                                   int32_t* __restrict__ idx) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * TOPK_WARPS + warp;
+  if (row >= rows) return;
+  const float* s = scores + (size_t)row * nk;
+  uint32_t key[NPL];
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) {
+    const int j = u * 32 + lane;
+    key[u] = j < nk ? order_key(s[j]) : 0u;      // padding keys sit below every real key
+  }
+  uint32_t T = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int u = 0; u < NPL; ++u) cnt += key[u] >= cand;
+    if ((int)__reduce_add_sync(0xffffffffu, cnt) >= k) T = cand;
+  }
+  uint32_t gtc = 0;
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) gtc += key[u] > T;
+  const int need = k - (int)__reduce_add_sync(0xffffffffu, gtc);   // keys equal to T that are kept
+  const uint32_t lt = (1u << lane) - 1u;
+  int eq_seen = 0, pos = 0;
+#pragma unroll
+  for (int u = 0; u < NPL; ++u) {
+    const int j = u * 32 + lane;
+    const bool in = j < nk;
+    const bool is_gt = in && key[u] > T;
+    const bool is_eq = in && key[u] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = is_gt || (is_eq && (eq_seen + __popc(eqm & lt)) < need);
+    eq_seen += __popc(eqm);
+    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+    if (in) mask[(size_t)row * nk + j] = sel ? 1 : 0;
+    if (sel) idx[(size_t)row * k + pos + __popc(selm & lt)] = j;
+    pos += __popc(selm);
+  }
+}
+
 // SoftTop-k of one logit row per warp (SLA2 detail page §4, Eq. 17): P_c = row
 // softmax of the logits, m_j = sigmoid(P_c[j] / tau + lambda) with lambda found
 // by bisection on [logit(k / nk) - 1 / tau, logit(k / nk)] so that the row sums
@@ -430,6 +476,23 @@ int scores_topk_max_nk() { return TOPK_MAX_NK; }
 
 cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st) {
   const int rows = s.BH * s.nq;
+  const dim3 grid((rows + TOPK_WARPS - 1) / TOPK_WARPS), block(TOPK_WARPS * 32);
+  if (s.nk <= 128) {
+    topk_reg_kernel<4><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    return cudaGetLastError();
+  }
+  if (s.nk <= 256) {
+    topk_reg_kernel<8><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    return cudaGetLastError();
+  }
+  if (s.nk <= 512) {
+    topk_reg_kernel<16><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    return cudaGetLastError();
+  }
+  if (s.nk <= 1024) {
+    topk_reg_kernel<32><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)TOPK_WARPS * s.nk * sizeof(uint32_t);
   cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   topk_kernel<<<(rows + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(scores, rows, s.nk, s.k, mask,
