@@ -377,7 +377,30 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
         f2_unpack(f2_add(rs2a, rs2b), ra0, ra1);
         l = l * corr + (ra0 + ra1);
         m = m_new;
-        // O must be rescaled by corr (after PV n-1 has finished) before PV n adds to it
+        // P buffer b was last read by PV g-2
+        if (g >= 2) {
+          ok = mbar_wait(p_free + b, ((g >> 1) - 1) & 1, abortf, a.status, a.budget_ns);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
+        if (QUANT) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int pc = ch ^ ((r >> 1) & 3);        // 64-byte swizzle
+            *reinterpret_cast<uint4*>(prow + pc * 16) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int pc = ch ^ (r & 7);               // 128-byte swizzle
+            *reinterpret_cast<uint4*>(prow + pc * 16) =
+                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        // O must be rescaled by corr (after PV n-1 has finished) before PV n adds to it;
+        // P is already stored, so its write and proxy fence overlap this wait
         if (n >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
           ok = mbar_wait(p_free + ((g - 1) & 1), ((g - 1) >> 1) & 1, abortf, a.status, a.budget_ns);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -419,31 +442,9 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
           }
           tmem_wait_st();
         }
-        // P buffer b was last read by PV g-2
-        if (g >= 2) {
-          ok = mbar_wait(p_free + b, ((g >> 1) - 1) & 1, abortf, a.status, a.budget_ns);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        }
-        uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
-        if (QUANT) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int pc = ch ^ ((r >> 1) & 3);        // 64-byte swizzle
-            *reinterpret_cast<uint4*>(prow + pc * 16) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          }
-        } else {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int pc = ch ^ (r & 7);               // 128-byte swizzle
-            *reinterpret_cast<uint4*>(prow + pc * 16) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          }
-        }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + b);
+        if (lane == 0) mbar_arrive(p_full + b);     // P written and O rescaled
       }
       if (!ok) break;
       // ---- item done: normalise O and store it, then hand O back to the MMA issuer
