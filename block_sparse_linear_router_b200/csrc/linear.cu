@@ -49,8 +49,10 @@ struct LinCfg {
   static constexpr int EG = D / 8;                     // feature groups of 8 per token row
   static constexpr int TG = LIN_CONV / EG;             // token groups
   static constexpr int TPT = BKB / TG;                 // tokens per converter thread
-  static constexpr int OFF_RED = 2 * STAGE;            // z partials [2][TG][D] + amax [2][8]
-  static constexpr int OFF_BAR = OFF_RED + (2 * TG * D + 16) * 4;
+  static constexpr int OFF_RED = 2 * STAGE;            // z partials [TG][D] + amax [2][8]
+  static constexpr int OFF_H = ((OFF_RED + (TG * D + 16) * 4) + 1023) / 1024 * 1024;   // staged h_j tile
+  static constexpr int H_BYTES = D * D * 2;
+  static constexpr int OFF_BAR = OFF_H + H_BYTES;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;
   static constexpr uint32_t IDESC = make_idesc_mn(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
   static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
@@ -72,6 +74,20 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
 // named barrier over the 256 converter threads (warps 0-7)
 __device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// Barrier over the 256 converter threads that returns, to every one of them,
+// whether any of them passed `failed`, so that all take the same exit and no
+// later barrier waits for a warp that has left.
+__device__ __forceinline__ bool conv_sync_any(bool failed) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)failed)
+      : "memory");
+  return r != 0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __grid_constant__ CUtensorMap tk,
                                                                       const __grid_constant__ CUtensorMap tv,
@@ -80,8 +96,9 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
   using C = LinCfg<D>;
   extern __shared__ uint8_t lsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
-  float* zred_all = reinterpret_cast<float*>(base + C::OFF_RED);     // [2][TG][D]
-  float* ared_all = zred_all + 2 * C::TG * D;                        // [2][8]
+  float* zred_all = reinterpret_cast<float*>(base + C::OFF_RED);     // [TG][D]
+  float* ared_all = zred_all + C::TG * D;                            // [2][8]
+  uint8_t* hst = base + C::OFF_H;                                    // h_j tile (h_mode 2), atom layout
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
   uint64_t* tma_full = bar;          // [2]
   uint64_t* conv_done = bar + 2;
@@ -203,8 +220,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     // accumulator released to the next block's MMA, then fp16 / bf16 / fp32 -> global
     auto readout = [&](int nn) -> bool {
       const int j = j0 + nn;
-      bool rok = mbar_wait(mma_done, nn & 1, abort_flag, o.status, o.budget_ns);
-      if (!__all_sync(0xffffffffu, rok)) return false;
+      const bool rok = mbar_wait(mma_done, nn & 1, abort_flag, o.status, o.budget_ns);
+      if (conv_sync_any(!rok)) return false;
       tc_fence_after();
       const int c = qd * 32 + lane;
       uint32_t rr[RC / 32][32];
@@ -215,22 +232,40 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       }
       tc_fence_before();
       mbar_arrive(rd_done);
-      if (qd * 32 < D) {
+      if (o.h_mode == 2 && qd * 32 < D) {
+        // -s h_j^T through shared memory: warps qd and qd + 4 own rows 32 qd .. 32 qd + 31,
+        // which form one contiguous 32 d x 2-byte piece of the atom layout; lane 0 of warp
+        // qd writes that piece to global memory with one bulk copy
+        const bool issuer = hh == 0 && lane == 0;
+        const uint32_t piece = (uint32_t)qd * 32 * D * 2;
+        if (issuer) bulk_wait_read0();      // its previous copy has read the staging rows
+        named_bar_sync(2 + qd, 64);
+        const float ns = -hs;
+#pragma unroll
+        for (int c2 = 0; c2 < RC / 32; ++c2) {
+          const int cc = hh * (RC / 32) + c2;
+          const uint32_t (&r)[32] = rr[c2];
+#pragma unroll
+          for (int q = 0; q < 32; q += 8)
+            *reinterpret_cast<uint4*>(hst + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
+                h2_bits(ns * __uint_as_float(r[q]), ns * __uint_as_float(r[q + 1])),
+                h2_bits(ns * __uint_as_float(r[q + 2]), ns * __uint_as_float(r[q + 3])),
+                h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
+                h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2 + qd, 64);
+        if (issuer) {
+          uint8_t* tile = static_cast<uint8_t*>(o.h) + ((size_t)bh * nk + j) * (size_t)(D * D * 2);
+          bulk_store(tile + piece, hst + piece, 32 * D * 2);
+          bulk_commit();
+        }
+      } else if (qd * 32 < D) {
 #pragma unroll
         for (int c2 = 0; c2 < RC / 32; ++c2) {
           const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
           const uint32_t (&r)[32] = rr[c2];
-          if (o.h_mode == 2) {
-            uint8_t* tile = static_cast<uint8_t*>(o.h) + ((size_t)bh * nk + j) * (size_t)(D * D * 2);
-            const float ns = -hs;
-#pragma unroll
-            for (int q = 0; q < 32; q += 8)
-              *reinterpret_cast<uint4*>(tile + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
-                  h2_bits(ns * __uint_as_float(r[q]), ns * __uint_as_float(r[q + 1])),
-                  h2_bits(ns * __uint_as_float(r[q + 2]), ns * __uint_as_float(r[q + 3])),
-                  h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
-                  h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
-          } else if (o.h_mode == 1) {
+          if (o.h_mode == 1) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
 #pragma unroll
             for (int q = 0; q < 32; q += 8)
@@ -254,10 +289,10 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     bool ok = true;
     for (int n = 0; n < cnt; ++n) {
       const int j = j0 + n;
-      float* zred = zred_all + (n & 1) * TG * D;
+      float* zred = zred_all;
       float* ared = ared_all + (n & 1) * 8;
       ok = mbar_wait(tma_full + (n & 1), (n >> 1) & 1, abort_flag, o.status, o.budget_ns);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      if (conv_sync_any(!ok)) { ok = false; break; }
       uint8_t* sK = base + (n & 1) * C::STAGE;
       uint8_t* sV = sK + C::OFF_V;
       const size_t rowbase = (size_t)bh * N + (size_t)j * BKB;
@@ -367,6 +402,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         }
       }
       // ---- operands complete: hand them (and the staged tile) to the MMA thread
+      if (!o.khat) conv_sync();   // the previous block's z partials have been summed (the quantised path synced above)
 #pragma unroll
       for (int c = 0; c < 8; ++c) zred[tg * D + eg * 8 + c] = zc[c];
       fence_proxy_async_smem();
@@ -404,6 +440,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       }
     }
     if (tid < D) o.zpart[((size_t)bh * G + chunk) * D + tid] = zp;
+    if (o.h_mode == 2) bulk_wait0();   // the staged tiles have reached global memory
   }
   tc_fence_before();
   __syncthreads();
