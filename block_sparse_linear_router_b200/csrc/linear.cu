@@ -180,13 +180,17 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
     const int tg = tid / EG;          // token group: tokens tg*TPT .. +TPT
     const int eg = tid % EG;          // feature / channel group: 8 columns eg*8 ..
     const int sl = eg >> 3, ch = eg & 7;
+    // V is converted with another split: each warp takes 32 / TG whole channel
+    // groups over all 64 tokens, so that a warp's V-hat^T stores fill whole rows
+    const int tgv = lane % TG, egv = warp * (32 / TG) + lane / TG;
+    const int slv = egv >> 3, chv = egv & 7;
     float cs[8], vinv[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       cs[c] = c32[(size_t)bh * D + eg * 8 + c];
       vinv[c] = 0.f;
       if (o.quant == 1) {
-        const float a = __uint_as_float(o.vamax[(size_t)bh * D + eg * 8 + c]);
+        const float a = __uint_as_float(o.vamax[(size_t)bh * D + egv * 8 + c]);
         vinv[c] = a > 0.f ? __fdiv_rn(448.f, a) : 0.f;
       }
     }
@@ -372,8 +376,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       float vv[TPT][8];
 #pragma unroll
       for (int u = 0; u < TPT; ++u) {
-        const int t = tg * TPT + u;
-        uint4* p = reinterpret_cast<uint4*>(sV + sl * C::SLAB + t * 128 + ((ch ^ (t & 7)) << 4));
+        const int t = tgv * TPT + u;
+        uint4* p = reinterpret_cast<uint4*>(sV + slv * C::SLAB + t * 128 + ((chv ^ (t & 7)) << 4));
         unpack8(*p, vv[u]);
         *p = make_uint4(h2_bits(vv[u][0], vv[u][1]), h2_bits(vv[u][2], vv[u][3]), h2_bits(vv[u][4], vv[u][5]),
                         h2_bits(vv[u][6], vv[u][7]));
@@ -381,19 +385,19 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       if (o.vhatT) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const size_t orow = ((size_t)bh * nk + j) * D + eg * 8 + c;
+          const size_t orow = ((size_t)bh * nk + j) * D + egv * 8 + c;
           if (o.quant == 1) {
             uint16_t pr[TPT / 2];
 #pragma unroll
             for (int u = 0; u < TPT; u += 2)
               pr[u / 2] = cvt_e4m3x2(__fmul_rn(vv[u][c], vinv[c]), __fmul_rn(vv[u + 1][c], vinv[c]));
-            uint8_t* vd = static_cast<uint8_t*>(o.vhatT) + orow * BKB + tg * TPT;
+            uint8_t* vd = static_cast<uint8_t*>(o.vhatT) + orow * BKB + tgv * TPT;
             if constexpr (TPT == 4)
               *reinterpret_cast<uint32_t*>(vd) = (uint32_t)pr[0] | ((uint32_t)pr[1] << 16);
             else
               *reinterpret_cast<uint16_t*>(vd) = pr[0];
           } else {
-            __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(o.vhatT) + orow * BKB + tg * TPT;
+            __nv_bfloat16* vd = static_cast<__nv_bfloat16*>(o.vhatT) + orow * BKB + tgv * TPT;
             if constexpr (TPT == 4)
               *reinterpret_cast<uint2*>(vd) = make_uint2(cvt_bf16x2(vv[0][c], vv[1][c]), cvt_bf16x2(vv[2][c], vv[3][c]));
             else
@@ -403,8 +407,10 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       }
       // ---- operands complete: hand them (and the staged tile) to the MMA thread
       if (!o.khat) conv_sync();   // the previous block's z partials have been summed (the quantised path synced above)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) zred[tg * D + eg * 8 + c] = zc[c];
+      // row tg of the z partials holds channels eg*8 .. +3 at eg*4 and eg*8+4 .. +7 at
+      // D/2 + eg*4 (two conflict-free 16-byte stores)
+      *reinterpret_cast<float4*>(zred + tg * D + eg * 4) = make_float4(zc[0], zc[1], zc[2], zc[3]);
+      *reinterpret_cast<float4*>(zred + tg * D + D / 2 + eg * 4) = make_float4(zc[4], zc[5], zc[6], zc[7]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(conv_done);
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       if (tid < D) {
         float z = 0.f;
 #pragma unroll
-        for (int g = 0; g < TG; ++g) z += zred[g * D + tid];
+        for (int g = 0; g < TG; ++g) z += zred[g * D + ((tid & 4) ? D / 2 : 0) + (tid >> 3) * 4 + (tid & 3)];
         o.z[((size_t)bh * nk + j) * D + tid] = z;
         zp += z;
       }

@@ -197,40 +197,54 @@ __global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restr
 }
 
 // Batched fp32 SIMT GEMM for the router's small products:
+// One or two batched fp32 products in one launch (blockIdx.z < p0.batch: p0,
+// else p1):
 //   C[b][m][n] = (sum_k X[b][m][k] * Y'[k][n]) / div
 // with Y' = Y[yb]^T (Y stored [N][K], "nt") or Y[yb] (stored [K][N], "nn"),
-// yb = b % ymod. K is the head dimension (a multiple of 32); each product is
-// accumulated sequentially over k in fp32. 64 x 64 tile per CTA, 4 x 4 per thread.
+// yb = b % ymod. K is the head dimension (a multiple of 16); each product is
+// accumulated sequentially over k in fp32. 64 x 64 tile per CTA of 128 threads,
+// 4 x 8 per thread, 16-deep k slabs: 8.5 KB of shared memory and at most 72
+// registers a thread, so that a CTA fits beside two linear-state CTAs on an SM.
+struct GemmProblem {
+  const float* X;
+  const float* Y;
+  float* C;
+  int batch, M, N, K, ymod;
+  float div;
+};
+
 template <bool NT>
-__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ X, const float* __restrict__ Y,
-                                                       float* __restrict__ C, int M, int N, int K, int ymod,
-                                                       float div) {
-  __shared__ __align__(16) float Xs[32][68];
-  __shared__ __align__(16) float Ys[32][68];
-  const int b = blockIdx.z, yb = b % ymod, tid = threadIdx.x;
+__global__ void __launch_bounds__(128, 7) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
+  __shared__ __align__(16) float Xs[16][68];
+  __shared__ __align__(16) float Ys[16][68];
+  const bool second = (int)blockIdx.z >= p0.batch;
+  const int b = second ? (int)blockIdx.z - p0.batch : (int)blockIdx.z;
+  const int M = second ? p1.M : p0.M, N = second ? p1.N : p0.N, K = second ? p1.K : p0.K;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  const int ty = tid >> 4, tx = tid & 15;
-  const float* Xb = X + (size_t)b * M * K;
-  const float* Yb = Y + (size_t)yb * N * K;
-  float acc[4][4];
+  if (m0 >= M || n0 >= N) return;
+  const int yb = b % (second ? p1.ymod : p0.ymod), tid = threadIdx.x;
+  const int ty = tid >> 3, tx = tid & 7;      // rows ty*4 .. +3, columns tx*4 .. +3 and 32 + tx*4 .. +3
+  const float* Xb = (second ? p1.X : p0.X) + (size_t)b * M * K;
+  const float* Yb = (second ? p1.Y : p0.Y) + (size_t)yb * N * K;
+  float acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += 32) {
-    // X tile: 64 rows x 32 k -> Xs[k][m]
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    // X tile: 64 rows x 16 k -> Xs[k][m]
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = tid + u * 256, r = t >> 3, kq = (t & 7) * 4;
+      const int t = tid + u * 128, r = t >> 2, kq = (t & 3) * 4;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (m0 + r < M) v = *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + r) * K + k0 + kq);
       Xs[kq][r] = v.x; Xs[kq + 1][r] = v.y; Xs[kq + 2][r] = v.z; Xs[kq + 3][r] = v.w;
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = tid + u * 256;
+      const int t = tid + u * 128;
       if (NT) {
-        const int r = t >> 3, kq = (t & 7) * 4;
+        const int r = t >> 2, kq = (t & 3) * 4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (n0 + r < N) v = *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq);
         Ys[kq][r] = v.x; Ys[kq + 1][r] = v.y; Ys[kq + 2][r] = v.z; Ys[kq + 3][r] = v.w;
@@ -242,26 +256,30 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
       }
     }
     __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
       const float4 a = *reinterpret_cast<const float4*>(&Xs[kk][ty * 4]);
-      const float4 bb = *reinterpret_cast<const float4*>(&Ys[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+      const float4 b0 = *reinterpret_cast<const float4*>(&Ys[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Ys[kk][32 + tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
   }
+  const float div = second ? p1.div : p0.div;
+  float* Cb = (second ? p1.C : p0.C) + (size_t)b * M * N;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = m0 + ty * 4 + i;
     if (m >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < N) C[((size_t)b * M + m) * N + n] = div == 1.f ? acc[i][j] : __fdiv_rn(acc[i][j], div);
+    for (int j = 0; j < 8; ++j) {
+      const int n = n0 + (j < 4 ? tx * 4 + j : 32 + tx * 4 + j - 4);
+      if (n < N) Cb[(size_t)m * N + n] = div == 1.f ? acc[i][j] : __fdiv_rn(acc[i][j], div);
     }
   }
 }
@@ -451,25 +469,26 @@ cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, floa
   return cudaGetLastError();
 }
 
-static cudaError_t gemm(bool nt, const float* X, const float* Y, float* C, int batch, int M, int N, int K, int ymod,
-                        float div, cudaStream_t st) {
-  dim3 grid((N + 63) / 64, (M + 63) / 64, batch);
+static cudaError_t gemm(bool nt, const GemmProblem& p0, const GemmProblem& p1, cudaStream_t st) {
+  const int N = p0.N > p1.N ? p0.N : p1.N, M = p0.M > p1.M ? p0.M : p1.M;
+  dim3 grid((N + 63) / 64, (M + 63) / 64, p0.batch + p1.batch);
   if (nt)
-    gemm_f32_kernel<true><<<grid, 256, 0, st>>>(X, Y, C, M, N, K, ymod, div);
+    gemm_f32_kernel<true><<<grid, 128, 0, st>>>(p0, p1);
   else
-    gemm_f32_kernel<false><<<grid, 256, 0, st>>>(X, Y, C, M, N, K, ymod, div);
+    gemm_f32_kernel<false><<<grid, 128, 0, st>>>(p0, p1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const float* kbar_s, const float* wq,
                         const float* wk, float* A, float* Bk, cudaStream_t st) {
-  cudaError_t e = gemm(false, qbar, wq, A, s.BH, s.nq, s.d, s.d, H, 1.f, st);
-  if (e != cudaSuccess) return e;
-  return gemm(false, kbar_s, wk, Bk, s.BH, s.nk, s.d, s.d, H, 1.f, st);
+  const GemmProblem pq{qbar, wq, A, s.BH, s.nq, s.d, s.d, H, 1.f};
+  const GemmProblem pk{kbar_s, wk, Bk, s.BH, s.nk, s.d, s.d, H, 1.f};
+  return gemm(false, pq, pk, st);
 }
 
 cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float* scores, cudaStream_t st) {
-  return gemm(true, A, Bk, scores, s.BH, s.nq, s.nk, s.d, s.BH, sqrtf((float)s.d), st);
+  const GemmProblem p{A, Bk, scores, s.BH, s.nq, s.nk, s.d, s.BH, sqrtf((float)s.d)};
+  return gemm(true, p, GemmProblem{nullptr, nullptr, nullptr, 0, 0, 0, 0, 1, 1.f}, st);
 }
 
 int scores_topk_max_nk() { return TOPK_MAX_NK; }
