@@ -196,15 +196,14 @@ __global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restr
   }
 }
 
-// Batched fp32 SIMT GEMM for the router's small products:
-// One or two batched fp32 products in one launch (blockIdx.z < p0.batch: p0,
-// else p1):
+// Batched fp32 SIMT GEMM for the router's small products, one or two of them
+// in one launch (blockIdx.z < p0.batch: p0, else p1):
 //   C[b][m][n] = (sum_k X[b][m][k] * Y'[k][n]) / div
 // with Y' = Y[yb]^T (Y stored [N][K], "nt") or Y[yb] (stored [K][N], "nn"),
 // yb = b % ymod. K is the head dimension (a multiple of 16); each product is
 // accumulated sequentially over k in fp32. 64 x 64 tile per CTA of 128 threads,
-// 4 x 8 per thread, 16-deep k slabs: 8.5 KB of shared memory and at most 72
-// registers a thread, so that a CTA fits beside two linear-state CTAs on an SM.
+// 4 x 8 per thread, 16-deep k slabs double-buffered in shared memory with the
+// next slab's global loads in flight during the current slab's products.
 struct GemmProblem {
   const float* X;
   const float* Y;
@@ -214,9 +213,9 @@ struct GemmProblem {
 };
 
 template <bool NT>
-__global__ void __launch_bounds__(128, 7) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
-  __shared__ __align__(16) float Xs[16][68];
-  __shared__ __align__(16) float Ys[16][68];
+__global__ void __launch_bounds__(128, 4) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
+  __shared__ __align__(16) float Xs[2][16][68];
+  __shared__ __align__(16) float Ys[2][16][68];
   const bool second = (int)blockIdx.z >= p0.batch;
   const int b = second ? (int)blockIdx.z - p0.batch : (int)blockIdx.z;
   const int M = second ? p1.M : p0.M, N = second ? p1.N : p0.N, K = second ? p1.K : p0.K;
@@ -226,41 +225,49 @@ __global__ void __launch_bounds__(128, 7) gemm_f32_kernel(GemmProblem p0, GemmPr
   const int ty = tid >> 3, tx = tid & 7;      // rows ty*4 .. +3, columns tx*4 .. +3 and 32 + tx*4 .. +3
   const float* Xb = (second ? p1.X : p0.X) + (size_t)b * M * K;
   const float* Yb = (second ? p1.Y : p0.Y) + (size_t)yb * N * K;
+  float4 px[2], py[2];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int t = tid + u * 128, r = t >> 2, kq = (t & 3) * 4;
+      px[u] = m0 + r < M ? *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + r) * K + k0 + kq)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (NT) {
+        py[u] = n0 + r < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const int kk = t >> 4, nq4 = (t & 15) * 4;
+        py[u] = n0 + nq4 < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(k0 + kk) * N + n0 + nq4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  };
   float acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    // X tile: 64 rows x 16 k -> Xs[k][m]
+  fetch(0);
+  for (int k0 = 0, buf = 0; k0 < K; k0 += 16, buf ^= 1) {
+    // X slab -> Xs[k][m], Y slab -> Ys[k][n]
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int t = tid + u * 128, r = t >> 2, kq = (t & 3) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m0 + r < M) v = *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + r) * K + k0 + kq);
-      Xs[kq][r] = v.x; Xs[kq + 1][r] = v.y; Xs[kq + 2][r] = v.z; Xs[kq + 3][r] = v.w;
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int t = tid + u * 128;
+      Xs[buf][kq][r] = px[u].x; Xs[buf][kq + 1][r] = px[u].y; Xs[buf][kq + 2][r] = px[u].z; Xs[buf][kq + 3][r] = px[u].w;
       if (NT) {
-        const int r = t >> 2, kq = (t & 3) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n0 + r < N) v = *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq);
-        Ys[kq][r] = v.x; Ys[kq + 1][r] = v.y; Ys[kq + 2][r] = v.z; Ys[kq + 3][r] = v.w;
+        Ys[buf][kq][r] = py[u].x; Ys[buf][kq + 1][r] = py[u].y; Ys[buf][kq + 2][r] = py[u].z; Ys[buf][kq + 3][r] = py[u].w;
       } else {
         const int kk = t >> 4, nq4 = (t & 15) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n0 + nq4 < N) v = *reinterpret_cast<const float4*>(Yb + (size_t)(k0 + kk) * N + n0 + nq4);
-        *reinterpret_cast<float4*>(&Ys[kk][nq4]) = v;
+        *reinterpret_cast<float4*>(&Ys[buf][kk][nq4]) = py[u];
       }
     }
-    __syncthreads();
+    __syncthreads();   // this slab is staged; every thread is done with the slab two steps back
+    if (k0 + 16 < K) fetch(k0 + 16);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&Xs[kk][ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Ys[kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Ys[kk][32 + tx * 4]);
+      const float4 a = *reinterpret_cast<const float4*>(&Xs[buf][kk][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Ys[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Ys[buf][kk][32 + tx * 4]);
       const float av[4] = {a.x, a.y, a.z, a.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -268,7 +275,6 @@ __global__ void __launch_bounds__(128, 7) gemm_f32_kernel(GemmProblem p0, GemmPr
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-    __syncthreads();
   }
   const float div = second ? p1.div : p0.div;
   float* Cb = (second ? p1.C : p0.C) + (size_t)b * M * N;
