@@ -16,7 +16,7 @@ using namespace sla2;
 
 namespace {
 
-constexpr unsigned long long DEFAULT_BUDGET_NS = 2000000000ull;   // 2 s per device wait
+constexpr unsigned long long DEFAULT_BUDGET_NS = kDefaultWaitBudgetNs;
 
 unsigned long long g_budget_ns = DEFAULT_BUDGET_NS;
 
@@ -159,7 +159,7 @@ sla2_status router_head(const sla2_desc* d, const Shape& s, const Layout& L, con
   if (v) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
   SLA2_TRY(launch_pool(s, q, k, v, at<float>(d, L.qbar), at<double>(d, L.ksum),
                        quant ? at<int8_t>(d, L.qhat) : nullptr, at<float>(d, L.sq),
-                       v ? at<unsigned>(d, L.vamax) : nullptr, st));
+                       v ? at<unsigned>(d, L.vamax) : nullptr, d->status, g_budget_ns, st));
   SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), at<float>(d, L.kbs),
                            st));
   return SLA2_OK;

@@ -24,8 +24,11 @@ struct Shape {
 // ---- router (router.cu) ----------------------------------------------------
 // Pass over Q, K (and V): pooled Q (fp32), exact fp64 column sums per key block,
 // optional INT8 Q-hat + s_q, optional per-channel |V| max (atomic, as uint bits).
+// Its pipeline waits are bounded by budget_ns (status gets the timeout code).
 cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void* v, float* qbar, double* ksum,
-                        int8_t* qhat, float* sq, unsigned* vamax, cudaStream_t st);
+                        int8_t* qhat, float* sq, unsigned* vamax, unsigned* status, unsigned long long budget_ns,
+                        cudaStream_t st);
+constexpr unsigned long long kDefaultWaitBudgetNs = 2000000000ull;   // 2 s per device wait
 // colmean (fp64 and fp32) from the per-block sums, and the smoothed pooled keys.
 cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, float* kbar_s,
                            cudaStream_t st);

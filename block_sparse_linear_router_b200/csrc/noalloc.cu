@@ -109,7 +109,8 @@ extern "C" sla2_status sla2_router_noalloc(const sla2_desc* desc, const void* q,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(p + off); };
   auto f64 = [&](size_t off) { return reinterpret_cast<double*>(p + off); };
-  if (sla2::launch_pool(s, q, k, nullptr, f32(L.qbar), f64(L.ksum), nullptr, nullptr, nullptr, st) != cudaSuccess)
+  if (sla2::launch_pool(s, q, k, nullptr, f32(L.qbar), f64(L.ksum), nullptr, nullptr, nullptr, nullptr,
+                        sla2::kDefaultWaitBudgetNs, st) != cudaSuccess)
     return SLA2_ERR_CUDA;
   if (sla2::launch_colmean(s, f64(L.ksum), f64(L.c64), f32(L.c32), f32(L.kbs), st) != cudaSuccess)
     return SLA2_ERR_CUDA;

@@ -27,142 +27,228 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
 }
 
-__device__ __forceinline__ float block_max_256(float v, float* red8) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int w = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red8[w] = v;
-  __syncthreads();
-  float m = red8[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) m = fmaxf(m, red8[i]);
-  return m;
-}
-
 // Symmetric INT8 of one value given the block's amax (fp32, RNE, no FMA).
 __device__ __forceinline__ int quant_i8(float x, float inv) {
   int qv = __float2int_rn(__fmul_rn(x, inv));
   return max(-127, min(127, qv));
 }
 
+constexpr int POOL_CONS = 256;                    // consumer threads (8 warps)
+constexpr int POOL_THREADS = POOL_CONS + 32;      // + one producer warp
+
 template <int D>
-__global__ void __launch_bounds__(256, 2) pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                   const __nv_bfloat16* __restrict__ k,
-                                                   const __nv_bfloat16* __restrict__ v, int N, int nq, int nk,
-                                                   float* __restrict__ qbar, double* __restrict__ ksum,
-                                                   int8_t* __restrict__ qhat, float* __restrict__ sq,
-                                                   unsigned* __restrict__ vamax) {
-  constexpr int TPR = D / 8;       // threads per row, 8 channels each
-  constexpr int RPP = 256 / TPR;   // rows per pass
-  constexpr int NP = BQ / RPP;     // passes over the 128 rows
-  __shared__ double red[RPP * D];
-  __shared__ float red8[8];
-  const int i = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const int cg = tid % TPR, rg = tid / TPR;
-  const size_t base = ((size_t)bh * N + (size_t)i * BQ) * D + cg * 8;
+struct PoolCfg {
+  static constexpr int TILE = BQ * D * 2;        // the 128 bf16 rows of one tensor for one query block
+  static constexpr int STAGE = 3 * TILE;         // Q, K, V
+  static constexpr int NS = D == 128 ? 2 : 4;    // pipeline depth (192 KB of stages)
+  static constexpr int TPR = D / 4;              // threads per row, 4 channels each
+  static constexpr int RPP = POOL_CONS / TPR;    // rows per pass
+  static constexpr int NP = BQ / RPP;            // passes over the 128 rows
+  static constexpr int RED = 8 * D;              // one per-warp partial table [8 warps][D]
+  static constexpr int OFF_RED = NS * STAGE;     // fp64 tables for Q, K rows 0..63, K rows 64..127; fp32 for V
+  static constexpr int OFF_A = OFF_RED + 3 * RED * 8 + RED * 4;   // per-warp |Q| maxima
+  static constexpr int OFF_BAR = OFF_A + 64;
+  static constexpr int SMEM = OFF_BAR + 2 * NS * 8 + 16;
+};
 
-  // V is read last: start bringing its rows into L2 now (one prefetch per 128-byte line)
-  if (vamax && (cg & 7) == 0) {
-#pragma unroll
-    for (int p = 0; p < NP; ++p)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(v + base + (size_t)(p * RPP + rg) * D)));
-  }
-  uint4 wq[NP], wk[NP];
-#pragma unroll
-  for (int p = 0; p < NP; ++p) wq[p] = __ldg(reinterpret_cast<const uint4*>(q + base + (size_t)(p * RPP + rg) * D));
-#pragma unroll
-  for (int p = 0; p < NP; ++p) wk[p] = __ldg(reinterpret_cast<const uint4*>(k + base + (size_t)(p * RPP + rg) * D));
+__device__ __forceinline__ void unpack4(const uint2& w, float (&x)[4]) {
+  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
+  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+}
 
-  // ---- Q: pooled mean (exact fp64 sum, one rounding to fp32) and INT8 Q-hat
-  double cs[8];
-  float amax = 0.f;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) cs[c] = 0.0;
-#pragma unroll
-  for (int p = 0; p < NP; ++p) {
-    float x[8];
-    unpack8(wq[p], x);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      cs[c] += (double)x[c];
-      amax = fmaxf(amax, fabsf(x[c]));
+// The INT8 code of RN(x * inv) rounded to nearest-even, in the low byte of the
+// result: adding 1.5 * 2^23 to a float of magnitude below 2^22 rounds it to an
+// integer whose two's complement occupies the low mantissa bits (the classic
+// magic-number conversion). |RN(x * inv)| <= 127 + 2^-17 when |x| <= a and
+// inv = RN(127 / a) is finite, so the code never leaves [-127, 127].
+__device__ __forceinline__ uint32_t q8_magic(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.f));
+}
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Barrier over the 256 consumer threads that returns, to every one of them,
+// whether any of them passed `failed` (so that all take the same exit).
+__device__ __forceinline__ bool pool_sync_any(bool failed) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)failed)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void pool_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Persistent pass over the query blocks (one CTA per SM). A producer warp
+// streams each block's 128 rows of Q, K (and V) into shared memory with three
+// bulk copies, two blocks ahead of the 8 consumer warps, which reduce them
+// there; the rows are contiguous in [B*H][N][d], so every copy is one piece.
+template <int D>
+__global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                               const __nv_bfloat16* __restrict__ k,
+                                                               const __nv_bfloat16* __restrict__ v, int BH, int N,
+                                                               int nq, int nk, float* __restrict__ qbar,
+                                                               double* __restrict__ ksum, int8_t* __restrict__ qhat,
+                                                               float* __restrict__ sq, unsigned* __restrict__ vamax,
+                                                               unsigned* status, unsigned long long budget_ns) {
+  using C = PoolCfg<D>;
+  constexpr int TPR = C::TPR, RPP = C::RPP, NP = C::NP, NS = C::NS;
+  extern __shared__ __align__(128) uint8_t pool_smem[];
+  uint8_t* base = pool_smem;
+  double* redq = reinterpret_cast<double*>(base + C::OFF_RED);
+  double* redk0 = redq + C::RED;
+  double* redk1 = redk0 + C::RED;
+  float* redv = reinterpret_cast<float*>(redk1 + C::RED);
+  float* reda = reinterpret_cast<float*>(base + C::OFF_A);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint64_t* empty = full + NS;
+  int* abort_flag = reinterpret_cast<int*>(empty + NS);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int items = BH * nq;
+  const uint32_t bytes = (v ? 3u : 2u) * (uint32_t)C::TILE;
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, POOL_CONS / 32);
     }
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) red[rg * D + cg * 8 + c] = cs[c];
   __syncthreads();
-  if (tid < D) {
-    double s = 0.0;
-    for (int r = 0; r < RPP; ++r) s += red[r * D + tid];
-    qbar[((size_t)bh * nq + i) * D + tid] = (float)(s / (double)BQ);
-  }
-  if (qhat) {
-    const float a = block_max_256(amax, red8);
-    const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      float x[8];
-      unpack8(wq[p], x);
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) lo |= (uint32_t)(quant_i8(x[c], inv) & 0xFF) << (8 * c);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) hi |= (uint32_t)(quant_i8(x[c + 4], inv) & 0xFF) << (8 * c);
-      *reinterpret_cast<uint2*>(qhat + base + (size_t)(p * RPP + rg) * D) = make_uint2(lo, hi);
+
+  if (warp == POOL_CONS / 32) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int n = 0;
+      for (int it = blockIdx.x; it < items; it += gridDim.x, ++n) {
+        const int s = n % NS;
+        if (n >= NS && !mbar_wait(empty + s, ((n / NS) & 1) ^ 1, abort_flag, status, budget_ns)) break;
+        const int bh = it / nq, i = it % nq;
+        const size_t row0 = ((size_t)bh * N + (size_t)i * BQ) * D;
+        uint8_t* st = base + s * C::STAGE;
+        mbar_arrive_expect_tx(full + s, bytes);
+        bulk_load(st, q + row0, C::TILE, full + s);
+        bulk_load(st + C::TILE, k + row0, C::TILE, full + s);
+        if (v) bulk_load(st + 2 * C::TILE, v + row0, C::TILE, full + s);
+      }
+      // copies still in flight after an abort land before the CTA exits
+      for (int j = n - NS < 0 ? 0 : n - NS; j < n; ++j) mbar_wait_drain(full + j % NS, (j / NS) & 1, budget_ns);
     }
-    if (tid == 0) sq[(size_t)bh * nq + i] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
+    return;
   }
 
-  // ---- K: exact fp64 column sums of the two 64-token key blocks
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) cs[c] = 0.0;
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      if ((p * RPP) / BKB != half) continue;
-      float x[8];
-      unpack8(wk[p], x);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) cs[c] += (double)x[c];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int c = 0; c < 8; ++c) red[rg * D + cg * 8 + c] = cs[c];
-    __syncthreads();
-    if (tid < D) {
-      double s = 0.0;
-      for (int r = 0; r < RPP; ++r) s += red[r * D + tid];
-      ksum[((size_t)bh * nk + 2 * i + half) * D + tid] = s;
-    }
-  }
+  // -------------------------------------------------------------------- consumers
+  const int cg = tid % TPR, rg = tid / TPR;   // channels cg*4 .. +3; rows rg, rg + RPP, ...
+  int n = 0;
+  for (int it = blockIdx.x; it < items; it += gridDim.x, ++n) {
+    const int s = n % NS;
+    const bool ok = mbar_wait(full + s, (n / NS) & 1, abort_flag, status, budget_ns);
+    // also: every consumer is done with the previous block's partial tables
+    if (pool_sync_any(!ok)) break;
+    const int bh = it / nq, i = it % nq;
+    const uint8_t* sQ = base + s * C::STAGE;
+    const uint8_t* sK = sQ + C::TILE;
+    const uint8_t* sV = sK + C::TILE;
 
-  // ---- V: per-channel |V| maximum (non-negative floats order like their bits)
-  if (vamax) {
-    uint4 wv[NP];
+    // ---- partial sums (exact in fp64) and maxima over this thread's rows
+    double cq[4], ck0[4], ck1[4];
+    float vm[4], amax = 0.f;
 #pragma unroll
-    for (int p = 0; p < NP; ++p) wv[p] = __ldg(reinterpret_cast<const uint4*>(v + base + (size_t)(p * RPP + rg) * D));
-    float vm[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) vm[c] = 0.f;
+    for (int c = 0; c < 4; ++c) {
+      cq[c] = 0.0; ck0[c] = 0.0; ck1[c] = 0.0; vm[c] = 0.f;
+    }
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      float x[8];
-      unpack8(wv[p], x);
+      const int row = p * RPP + rg;
+      float x[4], y[4];
+      unpack4(*reinterpret_cast<const uint2*>(sQ + row * D * 2 + cg * 8), x);
+      unpack4(*reinterpret_cast<const uint2*>(sK + row * D * 2 + cg * 8), y);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) vm[c] = fmaxf(vm[c], fabsf(x[c]));
+      for (int c = 0; c < 4; ++c) {
+        cq[c] += (double)x[c];
+        amax = fmaxf(amax, fabsf(x[c]));
+        if ((p * RPP) / BKB == 0) ck0[c] += (double)y[c];
+        else ck1[c] += (double)y[c];
+      }
+      if (v) {
+        unpack4(*reinterpret_cast<const uint2*>(sV + row * D * 2 + cg * 8), x);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vm[c] = fmaxf(vm[c], fabsf(x[c]));
+      }
     }
-    float* fred = reinterpret_cast<float*>(red);
-    __syncthreads();
+    // ---- combine the row groups of a warp (lanes with the same cg), then one row per warp
 #pragma unroll
-    for (int c = 0; c < 8; ++c) fred[rg * D + cg * 8 + c] = vm[c];
-    __syncthreads();
+    for (int o = TPR; o < 32; o <<= 1) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        cq[c] += __shfl_xor_sync(0xffffffffu, cq[c], o);
+        ck0[c] += __shfl_xor_sync(0xffffffffu, ck0[c], o);
+        ck1[c] += __shfl_xor_sync(0xffffffffu, ck1[c], o);
+        vm[c] = fmaxf(vm[c], __shfl_xor_sync(0xffffffffu, vm[c], o));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane < TPR) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        redq[warp * D + cg * 4 + c] = cq[c];
+        redk0[warp * D + cg * 4 + c] = ck0[c];
+        redk1[warp * D + cg * 4 + c] = ck1[c];
+        redv[warp * D + cg * 4 + c] = vm[c];
+      }
+    }
+    if (lane == 0) reda[warp] = amax;
+    pool_sync();
+
+    // ---- per-channel results (fixed order over the 8 warps; the fp64 sums are exact)
     if (tid < D) {
+      double sqs = 0.0, s0 = 0.0, s1 = 0.0;
       float m = 0.f;
-      for (int r = 0; r < RPP; ++r) m = fmaxf(m, fred[r * D + tid]);
-      atomicMax(vamax + (size_t)bh * D + tid, __float_as_uint(m));
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        sqs += redq[w * D + tid];
+        s0 += redk0[w * D + tid];
+        s1 += redk1[w * D + tid];
+        m = fmaxf(m, redv[w * D + tid]);
+      }
+      qbar[((size_t)bh * nq + i) * D + tid] = (float)(sqs / (double)BQ);
+      ksum[((size_t)bh * nk + 2 * i) * D + tid] = s0;
+      ksum[((size_t)bh * nk + 2 * i + 1) * D + tid] = s1;
+      if (v) atomicMax(vamax + (size_t)bh * D + tid, __float_as_uint(m));   // non-negative floats order like their bits
     }
+    // ---- INT8 Q-hat with the block's |Q| maximum
+    if (qhat) {
+      float a = reda[0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) a = fmaxf(a, reda[w]);
+      const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+      const size_t base_row = (size_t)bh * N + (size_t)i * BQ;
+      const bool magic = __float_as_uint(inv) < 0x7F800000u;   // finite (block-uniform); else the saturating path
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const int row = p * RPP + rg;
+        float x[4];
+        unpack4(*reinterpret_cast<const uint2*>(sQ + row * D * 2 + cg * 8), x);
+        uint32_t w;
+        if (magic) {
+          w = pack_low_bytes(q8_magic(x[0], inv), q8_magic(x[1], inv), q8_magic(x[2], inv), q8_magic(x[3], inv));
+        } else {
+          w = 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) w |= (uint32_t)(quant_i8(x[c], inv) & 0xFF) << (8 * c);
+        }
+        *reinterpret_cast<uint32_t*>(qhat + (base_row + row) * D + cg * 4) = w;
+      }
+      if (tid == 0) sq[(size_t)bh * nq + i] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
+    }
+    // ---- the stage is free for the producer
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + s);
   }
 }
 
@@ -201,8 +287,8 @@ __global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restr
 //   C[b][m][n] = (sum_k X[b][m][k] * Y'[k][n]) / div
 // with Y' = Y[yb]^T (Y stored [N][K], "nt") or Y[yb] (stored [K][N], "nn"),
 // yb = b % ymod. K is the head dimension (a multiple of 16); each product is
-// accumulated sequentially over k in fp32. 64 x 64 tile per CTA of 128 threads,
-// 4 x 8 per thread, 16-deep k slabs double-buffered in shared memory with the
+// accumulated sequentially over k in fp32. 32 x 64 tile per CTA of 128 threads,
+// 4 x 4 per thread, 16-deep k slabs double-buffered in shared memory with the
 // next slab's global loads in flight during the current slab's products.
 struct GemmProblem {
   const float* X;
@@ -213,26 +299,28 @@ struct GemmProblem {
 };
 
 template <bool NT>
-__global__ void __launch_bounds__(128, 4) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
-  __shared__ __align__(16) float Xs[2][16][68];
+__global__ void __launch_bounds__(128, 8) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
+  __shared__ __align__(16) float Xs[2][16][36];
   __shared__ __align__(16) float Ys[2][16][68];
   const bool second = (int)blockIdx.z >= p0.batch;
   const int b = second ? (int)blockIdx.z - p0.batch : (int)blockIdx.z;
   const int M = second ? p1.M : p0.M, N = second ? p1.N : p0.N, K = second ? p1.K : p0.K;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int m0 = blockIdx.y * 32, n0 = blockIdx.x * 64;
   if (m0 >= M || n0 >= N) return;
   const int yb = b % (second ? p1.ymod : p0.ymod), tid = threadIdx.x;
-  const int ty = tid >> 3, tx = tid & 7;      // rows ty*4 .. +3, columns tx*4 .. +3 and 32 + tx*4 .. +3
+  const int ty = tid >> 4, tx = tid & 15;     // rows ty*4 .. +3, columns tx*4 .. +3
   const float* Xb = (second ? p1.X : p0.X) + (size_t)b * M * K;
   const float* Yb = (second ? p1.Y : p0.Y) + (size_t)yb * N * K;
-  float4 px[2], py[2];
+  const int xr = tid >> 2, xk = (tid & 3) * 4;   // this thread's X element group of a slab
+  float4 px, py[2];
   auto fetch = [&](int k0) {
+    px = m0 + xr < M ? *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + xr) * K + k0 + xk)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = tid + u * 128, r = t >> 2, kq = (t & 3) * 4;
-      px[u] = m0 + r < M ? *reinterpret_cast<const float4*>(Xb + (size_t)(m0 + r) * K + k0 + kq)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int t = tid + u * 128;
       if (NT) {
+        const int r = t >> 2, kq = (t & 3) * 4;
         py[u] = n0 + r < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
@@ -242,19 +330,20 @@ __global__ void __launch_bounds__(128, 4) gemm_f32_kernel(GemmProblem p0, GemmPr
       }
     }
   };
-  float acc[4][8];
+  float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   fetch(0);
   for (int k0 = 0, buf = 0; k0 < K; k0 += 16, buf ^= 1) {
     // X slab -> Xs[k][m], Y slab -> Ys[k][n]
+    Xs[buf][xk][xr] = px.x; Xs[buf][xk + 1][xr] = px.y; Xs[buf][xk + 2][xr] = px.z; Xs[buf][xk + 3][xr] = px.w;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int t = tid + u * 128, r = t >> 2, kq = (t & 3) * 4;
-      Xs[buf][kq][r] = px[u].x; Xs[buf][kq + 1][r] = px[u].y; Xs[buf][kq + 2][r] = px[u].z; Xs[buf][kq + 3][r] = px[u].w;
+      const int t = tid + u * 128;
       if (NT) {
+        const int r = t >> 2, kq = (t & 3) * 4;
         Ys[buf][kq][r] = py[u].x; Ys[buf][kq + 1][r] = py[u].y; Ys[buf][kq + 2][r] = py[u].z; Ys[buf][kq + 3][r] = py[u].w;
       } else {
         const int kk = t >> 4, nq4 = (t & 15) * 4;
@@ -266,14 +355,12 @@ __global__ void __launch_bounds__(128, 4) gemm_f32_kernel(GemmProblem p0, GemmPr
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
       const float4 a = *reinterpret_cast<const float4*>(&Xs[buf][kk][ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Ys[buf][kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Ys[buf][kk][32 + tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float4 bq = *reinterpret_cast<const float4*>(&Ys[buf][kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
   const float div = second ? p1.div : p0.div;
@@ -283,8 +370,8 @@ __global__ void __launch_bounds__(128, 4) gemm_f32_kernel(GemmProblem p0, GemmPr
     const int m = m0 + ty * 4 + i;
     if (m >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = n0 + (j < 4 ? tx * 4 + j : 32 + tx * 4 + j - 4);
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
       if (n < N) Cb[(size_t)m * N + n] = div == 1.f ? acc[i][j] : __fdiv_rn(acc[i][j], div);
     }
   }
@@ -348,7 +435,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
 // The same hard Top-k with the row held in registers (NPL keys per lane, row
 // lengths up to 32 NPL): one compare per key and one warp reduction per bit.
 template <int NPL>
-__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_reg_kernel(const float* __restrict__ scores, int rows, int nk,
+__global__ void __launch_bounds__(TOPK_WARPS * 32, 1) topk_reg_kernel(const float* __restrict__ scores, int rows, int nk,
                                                                    int k, uint8_t* __restrict__ mask,
                                                                    int32_t* __restrict__ idx) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -364,10 +451,10 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_reg_kernel(const float* 
   uint32_t T = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
-    uint32_t cnt = 0;
+    uint32_t c4[4] = {0u, 0u, 0u, 0u};   // four short count chains instead of one long one
 #pragma unroll
-    for (int u = 0; u < NPL; ++u) cnt += key[u] >= cand;
-    if ((int)__reduce_add_sync(0xffffffffu, cnt) >= k) T = cand;
+    for (int u = 0; u < NPL; ++u) c4[u & 3] += key[u] >= cand;
+    if ((int)__reduce_add_sync(0xffffffffu, (c4[0] + c4[1]) + (c4[2] + c4[3])) >= k) T = cand;
   }
   uint32_t gtc = 0;
 #pragma unroll
@@ -457,15 +544,23 @@ cudaError_t launch_soft_topk(const Shape& s, const float* scores, float tau, flo
 }
 
 cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void* v, float* qbar, double* ksum,
-                        int8_t* qhat, float* sq, unsigned* vamax, cudaStream_t st) {
-  dim3 grid(s.nq, s.BH);
+                        int8_t* qhat, float* sq, unsigned* vamax, unsigned* status, unsigned long long budget_ns,
+                        cudaStream_t st) {
+  constexpr int kSMs = 148;   // B200 streaming multiprocessors
+  const int items = s.BH * s.nq;
+  const int grid = items < kSMs ? items : kSMs;
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   auto vb = static_cast<const __nv_bfloat16*>(v);
-  if (s.d == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(qb, kb, vb, s.N, s.nq, s.nk, qbar, ksum, qhat, sq, vamax);
-  else
-    pool_kernel<64><<<grid, 256, 0, st>>>(qb, kb, vb, s.N, s.nq, s.nk, qbar, ksum, qhat, sq, vamax);
+  if (s.d == 128) {
+    cudaFuncSetAttribute(pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, PoolCfg<128>::SMEM);
+    pool_kernel<128><<<grid, POOL_THREADS, PoolCfg<128>::SMEM, st>>>(qb, kb, vb, s.BH, s.N, s.nq, s.nk, qbar, ksum,
+                                                                      qhat, sq, vamax, status, budget_ns);
+  } else {
+    cudaFuncSetAttribute(pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, PoolCfg<64>::SMEM);
+    pool_kernel<64><<<grid, POOL_THREADS, PoolCfg<64>::SMEM, st>>>(qb, kb, vb, s.BH, s.N, s.nq, s.nk, qbar, ksum,
+                                                                    qhat, sq, vamax, status, budget_ns);
+  }
   return cudaGetLastError();
 }
 
@@ -477,7 +572,7 @@ cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, floa
 
 static cudaError_t gemm(bool nt, const GemmProblem& p0, const GemmProblem& p1, cudaStream_t st) {
   const int N = p0.N > p1.N ? p0.N : p1.N, M = p0.M > p1.M ? p0.M : p1.M;
-  dim3 grid((N + 63) / 64, (M + 63) / 64, p0.batch + p1.batch);
+  dim3 grid((N + 63) / 64, (M + 31) / 32, p0.batch + p1.batch);
   if (nt)
     gemm_f32_kernel<true><<<grid, 128, 0, st>>>(p0, p1);
   else
