@@ -397,6 +397,18 @@ __device__ __forceinline__ float h_fp16_scale(float vabs_max, int N) {
   return ldexpf(1.f, 15 - e);
 }
 
+// The INT8 code of RN(x * inv) rounded to nearest-even, in the low byte of the
+// result: adding 1.5 * 2^23 to a float of magnitude below 2^22 rounds it to an
+// integer whose two's complement occupies the low mantissa bits (the classic
+// magic-number conversion). |RN(x * inv)| <= 127 + 2^-17 when |x| <= a and
+// inv = RN(127 / a) is finite, so the code never leaves [-127, 127].
+__device__ __forceinline__ uint32_t q8_magic(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.f));
+}
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

@@ -228,18 +228,15 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       if (conv_sync_any(!rok)) return false;
       tc_fence_after();
       const int c = qd * 32 + lane;
-      uint32_t rr[RC / 32][32];
-      if (qd * 32 < D) {
-#pragma unroll
-        for (int c2 = 0; c2 < RC / 32; ++c2) tmem_ld32(lane_taddr + (hh * (RC / 32) + c2) * 32, rr[c2]);
-        tmem_wait_ld();
+      if (qd * 32 >= D) {   // no accumulator lanes for this warp (D = 64)
+        tc_fence_before();
+        mbar_arrive(rd_done);
+        return true;
       }
-      tc_fence_before();
-      mbar_arrive(rd_done);
-      if (o.h_mode == 2 && qd * 32 < D) {
-        // -s h_j^T through shared memory: warps qd and qd + 4 own rows 32 qd .. 32 qd + 31,
-        // which form one contiguous 32 d x 2-byte piece of the atom layout; lane 0 of warp
-        // qd writes that piece to global memory with one bulk copy
+      if (o.h_mode == 2) {
+        // -s h_j^T through shared memory, one 32-column chunk at a time: warps qd and qd + 4
+        // own rows 32 qd .. 32 qd + 31, which form one contiguous 32 d x 2-byte piece of the
+        // atom layout; lane 0 of warp qd writes that piece to global memory with one bulk copy
         const bool issuer = hh == 0 && lane == 0;
         const uint32_t piece = (uint32_t)qd * 32 * D * 2;
         if (issuer) bulk_wait_read0();      // its previous copy has read the staging rows
@@ -248,7 +245,9 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
 #pragma unroll
         for (int c2 = 0; c2 < RC / 32; ++c2) {
           const int cc = hh * (RC / 32) + c2;
-          const uint32_t (&r)[32] = rr[c2];
+          uint32_t r[32];
+          tmem_ld32(lane_taddr + cc * 32, r);
+          tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; q += 8)
             *reinterpret_cast<uint4*>(hst + atom_off(c, cc * 32 + q, D / 64)) = make_uint4(
@@ -257,6 +256,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
                 h2_bits(ns * __uint_as_float(r[q + 4]), ns * __uint_as_float(r[q + 5])),
                 h2_bits(ns * __uint_as_float(r[q + 6]), ns * __uint_as_float(r[q + 7])));
         }
+        tc_fence_before();
+        mbar_arrive(rd_done);               // the accumulator is free for the next block's MMA
         fence_proxy_async_smem();
         named_bar_sync(2 + qd, 64);
         if (issuer) {
@@ -264,27 +265,33 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
           bulk_store(tile + piece, hst + piece, 32 * D * 2);
           bulk_commit();
         }
-      } else if (qd * 32 < D) {
+        return true;
+      }
+      uint32_t rr[RC / 32][32];
 #pragma unroll
-        for (int c2 = 0; c2 < RC / 32; ++c2) {
-          const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
-          const uint32_t (&r)[32] = rr[c2];
-          if (o.h_mode == 1) {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+      for (int c2 = 0; c2 < RC / 32; ++c2) tmem_ld32(lane_taddr + (hh * (RC / 32) + c2) * 32, rr[c2]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(rd_done);
 #pragma unroll
-            for (int q = 0; q < 32; q += 8)
-              *reinterpret_cast<uint4*>(dst + q) = make_uint4(
-                  cvt_bf16x2(__uint_as_float(r[q]), __uint_as_float(r[q + 1])),
-                  cvt_bf16x2(__uint_as_float(r[q + 2]), __uint_as_float(r[q + 3])),
-                  cvt_bf16x2(__uint_as_float(r[q + 4]), __uint_as_float(r[q + 5])),
-                  cvt_bf16x2(__uint_as_float(r[q + 6]), __uint_as_float(r[q + 7])));
-          } else {
-            float* dst = static_cast<float*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+      for (int c2 = 0; c2 < RC / 32; ++c2) {
+        const int cc = hh * (RC / 32) + c2;   // 32-column chunk of this warp's half
+        const uint32_t (&r)[32] = rr[c2];
+        if (o.h_mode == 1) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
 #pragma unroll
-            for (int q = 0; q < 32; q += 4)
-              *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
-                                                                __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
-          }
+          for (int q = 0; q < 32; q += 8)
+            *reinterpret_cast<uint4*>(dst + q) = make_uint4(
+                cvt_bf16x2(__uint_as_float(r[q]), __uint_as_float(r[q + 1])),
+                cvt_bf16x2(__uint_as_float(r[q + 2]), __uint_as_float(r[q + 3])),
+                cvt_bf16x2(__uint_as_float(r[q + 4]), __uint_as_float(r[q + 5])),
+                cvt_bf16x2(__uint_as_float(r[q + 6]), __uint_as_float(r[q + 7])));
+        } else {
+          float* dst = static_cast<float*>(o.h) + (((size_t)bh * nk + j) * D + c) * D + cc * 32;
+#pragma unroll
+          for (int q = 0; q < 32; q += 4)
+            *reinterpret_cast<float4*>(dst + q) = make_float4(__uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                                              __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]));
         }
       }
       return true;
@@ -323,15 +330,23 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         const float a = fmaxf(fmaxf(fmaxf(ared[0], ared[1]), fmaxf(ared[2], ared[3])),
                               fmaxf(fmaxf(ared[4], ared[5]), fmaxf(ared[6], ared[7])));
         const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+        const bool magic = __float_as_uint(inv) < 0x7F800000u;   // finite (block-uniform); else the saturating path
 #pragma unroll
         for (int u = 0; u < TPT; ++u) {
           uint32_t lo = 0, hi = 0;
+          if (magic) {
+            lo = pack_low_bytes(q8_magic(x[u][0], inv), q8_magic(x[u][1], inv), q8_magic(x[u][2], inv),
+                                q8_magic(x[u][3], inv));
+            hi = pack_low_bytes(q8_magic(x[u][4], inv), q8_magic(x[u][5], inv), q8_magic(x[u][6], inv),
+                                q8_magic(x[u][7], inv));
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c], inv))));
-            const int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c + 4], inv))));
-            lo |= (uint32_t)(q0 & 0xFF) << (8 * c);
-            hi |= (uint32_t)(q1 & 0xFF) << (8 * c);
+            for (int c = 0; c < 4; ++c) {
+              const int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c], inv))));
+              const int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(x[u][c + 4], inv))));
+              lo |= (uint32_t)(q0 & 0xFF) << (8 * c);
+              hi |= (uint32_t)(q1 & 0xFF) << (8 * c);
+            }
           }
           *reinterpret_cast<uint2*>(o.khat + (rowbase + tg * TPT + u) * D + eg * 8) = make_uint2(lo, hi);
         }

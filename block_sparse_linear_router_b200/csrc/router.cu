@@ -56,18 +56,6 @@ __device__ __forceinline__ void unpack4(const uint2& w, float (&x)[4]) {
   x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
 }
 
-// The INT8 code of RN(x * inv) rounded to nearest-even, in the low byte of the
-// result: adding 1.5 * 2^23 to a float of magnitude below 2^22 rounds it to an
-// integer whose two's complement occupies the low mantissa bits (the classic
-// magic-number conversion). |RN(x * inv)| <= 127 + 2^-17 when |x| <= a and
-// inv = RN(127 / a) is finite, so the code never leaves [-127, 127].
-__device__ __forceinline__ uint32_t q8_magic(float x, float inv) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.f));
-}
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
-
 // Barrier over the 256 consumer threads that returns, to every one of them,
 // whether any of them passed `failed` (so that all take the same exit).
 __device__ __forceinline__ bool pool_sync_any(bool failed) {
