@@ -98,10 +98,10 @@ def measured_traffic(name):
 
 
 def launches_per_forward(w, k):
-    """Kernels one forward launches: router 6 (pool, column means, two projections,
-    logits, top-k), linear state 2, sparse 1, Z_i 1 and epilogue 1 (no Z_i pass when
-    every key block is selected)."""
-    return 6 + 2 + 1 + (2 if k < w.N // 64 else 1)
+    """Kernels one forward launches: router 5 (pool, column means, both projections in
+    one launch, logits, top-k), linear state 2, sparse 1, Z_i 1 and epilogue 1 (no Z_i
+    pass when every key block is selected)."""
+    return 5 + 2 + 1 + (2 if k < w.N // 64 else 1)
 
 
 class ClockSampler:
