@@ -72,10 +72,11 @@ def work_model(w, k):
 # kernel source they were taken on: sha256 prefix of the kernel file + device.cuh + kernels.cuh.
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum, --set full capture
-    "sparse": ("sparse.cu", "4a052642555b5e87", 298.0e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
-    # dram__bytes.sum.per_second x gpu__time_duration.sum, section capture
-    "epilogue": ("epilogue.cu", "cbefc15d0eb99f09", 594.0e6, "ncu dram__bytes.sum.per_second x duration"),
-    "linear_state": ("linear.cu", "5e42d52ed190c7af", 472.0e6, "ncu dram__bytes.sum.per_second x duration"),
+    "sparse": ("sparse.cu", "7ec4498840bfcb5c", 298.1e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    # dram__bytes.sum.per_second x gpu__time_duration.sum, section captures
+    "epilogue": ("epilogue.cu", "37149c1017ff3577", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
+    "linear_state": ("linear.cu", "f63c8cad80d11430", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
+    "router": ("router.cu", "e08d9a519bfa4f1f", 345.8e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
 }
 
 
