@@ -20,13 +20,6 @@ namespace sla2 {
 
 namespace {
 
-__device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
-  x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
-  x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-  x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
-  x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
-}
-
 // Symmetric INT8 of one value given the block's amax (fp32, RNE, no FMA).
 __device__ __forceinline__ int quant_i8(float x, float inv) {
   int qv = __float2int_rn(__fmul_rn(x, inv));
@@ -270,10 +263,9 @@ __global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restr
   }
 }
 
-// Batched fp32 SIMT GEMM for the router's small products, one or two of them
-// in one launch (blockIdx.z < p0.batch: p0, else p1):
-//   C[b][m][n] = (sum_k X[b][m][k] * Y'[k][n]) / div
-// with Y' = Y[yb]^T (Y stored [N][K], "nt") or Y[yb] (stored [K][N], "nn"),
+// Batched fp32 SIMT GEMM for the router's projections, both of them in one
+// launch (blockIdx.z < p0.batch: p0, else p1):
+//   C[b][m][n] = (sum_k X[b][m][k] * Y[yb][k][n]) / div,  Y stored [K][N],
 // yb = b % ymod. K is the head dimension (a multiple of 16); each product is
 // accumulated sequentially over k in fp32. 32 x 64 tile per CTA of 128 threads,
 // 4 x 4 per thread, 16-deep k slabs double-buffered in shared memory with the
@@ -286,7 +278,6 @@ struct GemmProblem {
   float div;
 };
 
-template <bool NT>
 __global__ void __launch_bounds__(128, 8) gemm_f32_kernel(GemmProblem p0, GemmProblem p1) {
   __shared__ __align__(16) float Xs[2][16][36];
   __shared__ __align__(16) float Ys[2][16][68];
@@ -307,15 +298,9 @@ __global__ void __launch_bounds__(128, 8) gemm_f32_kernel(GemmProblem p0, GemmPr
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int t = tid + u * 128;
-      if (NT) {
-        const int r = t >> 2, kq = (t & 3) * 4;
-        py[u] = n0 + r < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(n0 + r) * K + k0 + kq)
+      const int kk = t >> 4, nq4 = (t & 15) * 4;
+      py[u] = n0 + nq4 < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(k0 + kk) * N + n0 + nq4)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        const int kk = t >> 4, nq4 = (t & 15) * 4;
-        py[u] = n0 + nq4 < N ? *reinterpret_cast<const float4*>(Yb + (size_t)(k0 + kk) * N + n0 + nq4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
     }
   };
   float acc[4][4];
@@ -330,13 +315,8 @@ __global__ void __launch_bounds__(128, 8) gemm_f32_kernel(GemmProblem p0, GemmPr
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int t = tid + u * 128;
-      if (NT) {
-        const int r = t >> 2, kq = (t & 3) * 4;
-        Ys[buf][kq][r] = py[u].x; Ys[buf][kq + 1][r] = py[u].y; Ys[buf][kq + 2][r] = py[u].z; Ys[buf][kq + 3][r] = py[u].w;
-      } else {
-        const int kk = t >> 4, nq4 = (t & 15) * 4;
-        *reinterpret_cast<float4*>(&Ys[buf][kk][nq4]) = py[u];
-      }
+      const int kk = t >> 4, nq4 = (t & 15) * 4;
+      *reinterpret_cast<float4*>(&Ys[buf][kk][nq4]) = py[u];
     }
     __syncthreads();   // this slab is staged; every thread is done with the slab two steps back
     if (k0 + 16 < K) fetch(k0 + 16);
@@ -361,6 +341,80 @@ __global__ void __launch_bounds__(128, 8) gemm_f32_kernel(GemmProblem p0, GemmPr
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
       if (n < N) Cb[(size_t)m * N + n] = div == 1.f ? acc[i][j] : __fdiv_rn(acc[i][j], div);
+    }
+  }
+}
+
+// Router logits s = A Bk^T / div for one head's 32 query blocks x 64 key blocks
+// per CTA, with the whole K = d extent staged once: rows of A and Bk are copied
+// 16 bytes at a time (cp.async, no register staging) into rows padded to d + 4
+// floats, then one barrier, then d sequential fp32 FMAs per output (the same
+// order as gemm_f32_kernel, so the logits are bit-identical). 128 threads, 4 x 4
+// outputs each: query rows ty*4 .. +3, key rows tx + 16 j (so that a warp's key
+// reads spread over the banks).
+template <int D>
+__global__ void __launch_bounds__(128) logits_fullk_kernel(const float* __restrict__ A, const float* __restrict__ Bk,
+                                                           float* __restrict__ C, int M, int N, float div) {
+  constexpr int LD = D + 4;   // padded row length (floats); rows stay 16-byte aligned
+  extern __shared__ __align__(16) float lg_smem[];
+  float* As = lg_smem;             // [32][LD]
+  float* Bs = lg_smem + 32 * LD;   // [64][LD]
+  const int b = blockIdx.z, m0 = blockIdx.y * 32, n0 = blockIdx.x * 64, tid = threadIdx.x;
+  const float* Ab = A + ((size_t)b * M) * D;
+  const float* Bb = Bk + ((size_t)b * N) * D;
+  constexpr int CPR = D / 4;   // 16-byte pieces per row
+  for (int p = tid; p < 32 * CPR; p += 128) {
+    const int r = p / CPR, q = p % CPR;
+    float* dst = As + r * LD + q * 4;
+    if (m0 + r < M)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                   "l"(Ab + (size_t)(m0 + r) * D + q * 4) : "memory");
+    else
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int p = tid; p < 64 * CPR; p += 128) {
+    const int r = p / CPR, q = p % CPR;
+    float* dst = Bs + r * LD + q * 4;
+    if (n0 + r < N)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                   "l"(Bb + (size_t)(n0 + r) * D + q * 4) : "memory");
+    else
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < D; k += 4) {
+    float4 a[4], bq[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(As + (ty * 4 + i) * LD + k);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bq[j] = *reinterpret_cast<const float4*>(Bs + (tx + 16 * j) * LD + k);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = fmaf(a[i].x, bq[j].x, acc[i][j]);
+        acc[i][j] = fmaf(a[i].y, bq[j].y, acc[i][j]);
+        acc[i][j] = fmaf(a[i].z, bq[j].z, acc[i][j]);
+        acc[i][j] = fmaf(a[i].w, bq[j].w, acc[i][j]);
+      }
+  }
+  float* Cb = C + (size_t)b * M * N;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n < N) Cb[(size_t)m * N + n] = __fdiv_rn(acc[i][j], div);
     }
   }
 }
@@ -558,13 +612,10 @@ cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, floa
   return cudaGetLastError();
 }
 
-static cudaError_t gemm(bool nt, const GemmProblem& p0, const GemmProblem& p1, cudaStream_t st) {
+static cudaError_t gemm(const GemmProblem& p0, const GemmProblem& p1, cudaStream_t st) {
   const int N = p0.N > p1.N ? p0.N : p1.N, M = p0.M > p1.M ? p0.M : p1.M;
   dim3 grid((N + 63) / 64, (M + 31) / 32, p0.batch + p1.batch);
-  if (nt)
-    gemm_f32_kernel<true><<<grid, 128, 0, st>>>(p0, p1);
-  else
-    gemm_f32_kernel<false><<<grid, 128, 0, st>>>(p0, p1);
+  gemm_f32_kernel<<<grid, 128, 0, st>>>(p0, p1);
   return cudaGetLastError();
 }
 
@@ -572,12 +623,21 @@ cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const float* k
                         const float* wk, float* A, float* Bk, cudaStream_t st) {
   const GemmProblem pq{qbar, wq, A, s.BH, s.nq, s.d, s.d, H, 1.f};
   const GemmProblem pk{kbar_s, wk, Bk, s.BH, s.nk, s.d, s.d, H, 1.f};
-  return gemm(false, pq, pk, st);
+  return gemm(pq, pk, st);
 }
 
 cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float* scores, cudaStream_t st) {
-  const GemmProblem p{A, Bk, scores, s.BH, s.nq, s.nk, s.d, s.BH, sqrtf((float)s.d)};
-  return gemm(true, p, GemmProblem{nullptr, nullptr, nullptr, 0, 0, 0, 0, 1, 1.f}, st);
+  const dim3 grid((s.nk + 63) / 64, (s.nq + 31) / 32, s.BH);
+  const float div = sqrtf((float)s.d);
+  if (s.d == 128) {
+    const int smem = 96 * (128 + 4) * 4;
+    cudaFuncSetAttribute(logits_fullk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    logits_fullk_kernel<128><<<grid, 128, smem, st>>>(A, Bk, scores, s.nq, s.nk, div);
+  } else {
+    const int smem = 96 * (64 + 4) * 4;
+    logits_fullk_kernel<64><<<grid, 128, smem, st>>>(A, Bk, scores, s.nq, s.nk, div);
+  }
+  return cudaGetLastError();
 }
 
 int scores_topk_max_nk() { return TOPK_MAX_NK; }
