@@ -76,7 +76,7 @@ MEASURED_TRAFFIC = {
     # dram__bytes.sum.per_second x gpu__time_duration.sum, section captures
     "epilogue": ("epilogue.cu", "37149c1017ff3577", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
     "linear_state": ("linear.cu", "f63c8cad80d11430", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "router": ("router.cu", "e08d9a519bfa4f1f", 345.8e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
+    "router": ("router.cu", "27189c8c7b5b2c71", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
 }
 
 
@@ -413,9 +413,9 @@ def main():
         "config": {"workload": f"{w.name} B={w.B} H={w.H} N={w.N} d={w.d} k%={w.topk_frac * 100:g} (k={k} of {w.nk})",
                    "l2": "no flush: Q/K/V 302 MB > 126 MB L2", "parallelism": f"replicas x{ws}"},
         "roofline": roofline, "kernels": kern,
-        "stages": "router = pass over Q/K/V + column means; linear_state = linear state + reduce, with the "
-                  "router's projections / logits / top-k concurrent on a second stream; sparse = sparse branch "
-                  "(Z_i concurrent); epilogue = linear apply + mix",
+        "stages": "router = pass over Q/K/V + column means; linear_state = linear state + reduce on a second "
+                  "stream, with the router's projections / logits / top-k concurrent on the caller's stream; "
+                  "sparse = sparse branch (Z_i concurrent); epilogue = linear apply + mix",
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_forward(w, k) * K, "clocks": clk,
         "sparse_issued_tops": kern["sparse"]["achieved"],

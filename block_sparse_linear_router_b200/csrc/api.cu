@@ -341,15 +341,15 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   if (r != SLA2_OK) return r;
   SLA2_TRY(mark(1));
 
-  // fork: the router's tail on the auxiliary stream, the linear state on `st`
+  // fork: the linear state on the auxiliary stream, the router's tail on `st`. The
+  // projection GEMM, enqueued on the GPU at the same time, takes the SMs first and
+  // runs at full width; the logits and the top-k then fit beside the linear-state
+  // CTAs and finish while it runs, so the sparse branch follows the linear state.
   std::lock_guard<std::mutex> aux_lock(g_aux_mu);
   AuxStream* aux = nullptr;
   SLA2_TRY(aux_stream(&aux));
   SLA2_TRY(cudaEventRecord(aux->fork, st));
   SLA2_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
-  r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, aux->stream);
-  if (r != SLA2_OK) return r;
-  SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
 
   LinearOut o{};
   o.h = at<void>(desc, L.h);
@@ -365,9 +365,12 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   o.quant = quant;
   o.status = desc->status;
   o.budget_ns = g_budget_ns;
-  SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
+  SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, aux->stream));
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, o.vamax, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
-                                at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), st));
+                                at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), aux->stream));
+  SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
+  r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, st);
+  if (r != SLA2_OK) return r;
   SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join
   SLA2_TRY(mark(2));
   // Z_i (needs the top-k and Z_total) on the auxiliary stream, concurrently with the sparse branch

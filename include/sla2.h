@@ -172,9 +172,10 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
 /* The whole forward pass (steps 1-4): out = alpha O_s + (1 - alpha) O_l.
  *   out : bf16 or fp32 (desc->out_dtype) [B][H][N][d]
  * All intermediates live in desc->workspace; optional debug exports in desc.
- * The router's projections, logits and top-k run on a library-owned
- * non-blocking stream, forked from and joined back into `stream` with events,
- * concurrently with the linear-state pass. That stream and its two events are
+ * The linear-state pass runs on a library-owned non-blocking stream, forked
+ * from and joined back into `stream` with events, concurrently with the
+ * router's projections, logits and top-k on `stream`; the Z_i pass runs on it
+ * too, concurrently with the sparse branch. That stream and its two events are
  * created by the first call on each device and kept until the process exits;
  * make that first call outside any stream capture. Later calls can be captured
  * (the fork and join become graph edges). Calls from several host threads are
