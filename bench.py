@@ -76,7 +76,7 @@ MEASURED_TRAFFIC = {
     # dram__bytes.sum.per_second x gpu__time_duration.sum, section captures
     "epilogue": ("epilogue.cu", "37149c1017ff3577", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
     "linear_state": ("linear.cu", "f63c8cad80d11430", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "router": ("router.cu", "27189c8c7b5b2c71", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
+    "router": ("router.cu", "9b35b2e1b1be3bac", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
 }
 
 

@@ -6,8 +6,9 @@
 //             block, and each channel's |V| maximum (for the FP8 V scale).
 //   colmean   c = (sum over all key blocks) / N in fp64; fp32 copy for K_s.
 //   proj      A = Qbar Wq, Bk = (Kbar - c) Wk  (y = x W, W stored [d_in][d_out]).
-//   topk      s_ij = A_i . Bk_j / sqrt(d) in fp32; per row the k largest,
-//             ties to the lower block index; mask M_c and ascending index list.
+//   logits    s_ij = A_i . Bk_j / sqrt(d) in fp32.
+//   topk      per row the k largest s_ij, ties to the lower block index; mask
+//             M_c and ascending index list (soft_topk: the SoftTop-k weights).
 //
 // HBM-bound: pool reads Q, K, V once (bf16) and writes Q-hat; the rest touches
 // O((nq + nk) d) bytes per head.
