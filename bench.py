@@ -46,7 +46,8 @@ def load_peaks():
 
 
 def work_model(w, k):
-    """Algorithmic work of one forward pass."""
+    """Algorithmic work of one forward pass: bytes of the HBM-bound stages, 8-bit ops
+    of the sparse branch and fp16 flops of the epilogue, per the definitions below."""
     B, H, N, d = w.B, w.H, w.N, w.d
     BH, nq, nk = B * H, N // 128, N // 64
     E = BH * N * d
