@@ -104,3 +104,32 @@ def test_soft_topk_temperature_multiplied_is_caught(monkeypatch):
         return orig(np.asarray(pc_row) * tau * tau, k, tau, iters)   # P_c * tau instead of P_c / tau
     monkeypatch.setattr(O, "soft_topk", wrong)
     assert _fails(pins.test_soft_topk_small_tau_is_hard_topk)
+
+
+def test_transposed_projection_is_caught(monkeypatch):
+    orig = O.router_scores
+
+    def wrong(Q, K, Wq, Wk, smooth=True):
+        return orig(Q, K, np.asarray(Wq).T, np.asarray(Wk).T, smooth)   # y = x W^T
+    monkeypatch.setattr(O, "router_scores", wrong)
+    assert _fails(pins.test_router_projection_orientation_elementary_matrices)
+
+
+def test_swapped_projections_are_caught(monkeypatch):
+    orig = O.router_scores
+
+    def wrong(Q, K, Wq, Wk, smooth=True):
+        return orig(Q, K, Wk, Wq, smooth)                               # proj_k applied to Q
+    monkeypatch.setattr(O, "router_scores", wrong)
+    assert _fails(pins.test_router_projection_orientation_elementary_matrices)
+
+
+def test_first_heads_projection_everywhere_is_caught(monkeypatch):
+    orig = O.router_scores
+    first = {}
+
+    def wrong(Q, K, Wq, Wk, smooth=True):
+        first.setdefault("w", (Wq, Wk))                                  # head 0's matrices reused
+        return orig(Q, K, first["w"][0], first["w"][1], smooth)
+    monkeypatch.setattr(O, "router_scores", wrong)
+    assert _fails(pins.test_router_uses_each_batch_and_heads_own_inputs)

@@ -144,6 +144,44 @@ def test_router_identity_projection_is_heuristic_router():
     np.testing.assert_allclose(O.compressed_probs(s), Pc_ref, rtol=1e-12, atol=1e-15)
 
 
+def test_router_projection_orientation_elementary_matrices():
+    """y = x W with W stored [d_in][d_out]: with proj_q = E(0 -> 1) and proj_k =
+    E(2 -> 1) (a single one at row 0 / row 2, column 1) the projected vectors meet
+    only in feature 1, so s_ij = Qbar_i[0] * Kbar_s,j[2] / sqrt(d). A transposed or
+    swapped projection moves the features elsewhere and fails this."""
+    inp = make_custom(1, 1, 512, 16, 0.25, seed=15)
+    Q, K, V, _, _, _ = _head(inp)
+    Wq = np.zeros((16, 16)); Wq[0, 1] = 1.0
+    Wk = np.zeros((16, 16)); Wk[2, 1] = 1.0
+    s = O.router_scores(Q, K, Wq, Wk)
+    Qt, Kt = torch.from_numpy(Q), torch.from_numpy(K)
+    Qb = Qt.reshape(4, 128, 16).mean(1)
+    Kb = (Kt - Kt.mean(0)).reshape(8, 64, 16).mean(1)
+    ref = torch.outer(Qb[:, 0], Kb[:, 2]).numpy() / 4.0
+    np.testing.assert_allclose(s, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_router_uses_each_batch_and_heads_own_inputs():
+    """The [B, H] router takes head h's projections and head (b, h)'s Q, K:
+    with elementary projections that differ per head (feature 0 of Q against
+    feature h + 1 of K_s), each head's logits equal the outer product computed
+    directly with torch pooling."""
+    inp = make_custom(2, 3, 512, 16, 0.25, seed=16)
+    H, d = 3, 16
+    Wq = np.zeros((H, d, d)); Wk = np.zeros((H, d, d))
+    for h in range(H):
+        Wq[h, 0, 5] = 1.0
+        Wk[h, h + 1, 5] = 1.0
+    _, _, scores = O.router(inp.q, inp.k, Wq, Wk, 0.25)
+    for b in range(2):
+        for h in range(H):
+            Qt, Kt = inp.q[b, h].double(), inp.k[b, h].double()
+            Qb = Qt.reshape(4, 128, d).mean(1)
+            Kb = (Kt - Kt.mean(0)).reshape(8, 64, d).mean(1)
+            ref = torch.outer(Qb[:, 0], Kb[:, h + 1]).numpy() / 4.0
+            np.testing.assert_allclose(scores[b, h], ref, rtol=1e-12, atol=1e-15)
+
+
 def test_topk_matches_bruteforce_sort_and_counts():
     rng = np.random.default_rng(6)
     s = rng.standard_normal((16, 40))
