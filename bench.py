@@ -73,11 +73,11 @@ def work_model(w, k):
 # kernel source they were taken on: sha256 prefix of the kernel file + device.cuh + kernels.cuh.
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum, --set full capture
-    "sparse": ("sparse.cu", "7ec4498840bfcb5c", 298.1e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    "sparse": ("sparse.cu", "3a73ccef7b0d189c", 298.1e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
     # dram__bytes.sum.per_second x gpu__time_duration.sum, section captures
-    "epilogue": ("epilogue.cu", "37149c1017ff3577", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "linear_state": ("linear.cu", "f63c8cad80d11430", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "router": ("router.cu", "9b35b2e1b1be3bac", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
+    "epilogue": ("epilogue.cu", "1b0cc1424c18eeed", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
+    "linear_state": ("linear.cu", "67c76cddfc1bdc85", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
+    "router": ("router.cu", "4eadfd52602acf06", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
 }
 
 

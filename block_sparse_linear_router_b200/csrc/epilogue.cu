@@ -72,6 +72,8 @@ struct EpiCfg {
   static constexpr int OFF_BAR = OFF_DEN + 4 * BQ * 4;
   static constexpr int NBAR = 2 * NS + 9;
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
+  static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
+  static_assert(STAGE % 1024 == 0 && OFF_Z % 16 == 0, "bulk-copy and swizzle-atom alignment of the ring");
   static constexpr int KSTEPS = D / 16;              // 16 fp16 (8 TMEM columns of A) per MMA
   static constexpr uint32_t ACOL = 256;              // A buffers: columns ACOL + b * D / 2
   static constexpr uint32_t TMEM_COLS = 512;

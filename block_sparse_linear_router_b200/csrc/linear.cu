@@ -54,6 +54,8 @@ struct LinCfg {
   static constexpr int H_BYTES = D * D * 2;
   static constexpr int OFF_BAR = OFF_H + H_BYTES;
   static constexpr int SMEM = OFF_BAR + 64 + 1024;
+  static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM (228 KB, 1 KB reserved per CTA)");
+  static_assert(OFF_H % 1024 == 0 && (32 * D * 2) % 16 == 0, "h staging: atom alignment, 16-byte bulk pieces");
   static constexpr uint32_t IDESC = make_idesc_mn(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, M = 128, N = D
   static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;
   static constexpr uint32_t COL_TOT = D;                // running partial H^T

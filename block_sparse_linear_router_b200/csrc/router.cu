@@ -43,6 +43,8 @@ struct PoolCfg {
   static constexpr int OFF_A = OFF_RED + 3 * RED * 8 + RED * 4;   // per-warp |Q| maxima
   static constexpr int OFF_BAR = OFF_A + 64;
   static constexpr int SMEM = OFF_BAR + 2 * NS * 8 + 16;
+  static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
+  static_assert(TILE % 16 == 0 && STAGE % 16 == 0 && OFF_BAR % 8 == 0, "bulk-copy and mbarrier alignment");
 };
 
 __device__ __forceinline__ void unpack4(const uint2& w, float (&x)[4]) {
@@ -357,6 +359,7 @@ template <int D>
 __global__ void __launch_bounds__(128) logits_fullk_kernel(const float* __restrict__ A, const float* __restrict__ Bk,
                                                            float* __restrict__ C, int M, int N, float div) {
   constexpr int LD = D + 4;   // padded row length (floats); rows stay 16-byte aligned
+  static_assert((LD * 4) % 16 == 0 && 96 * LD * 4 <= 232448, "cp.async row alignment, shared memory");
   extern __shared__ __align__(16) float lg_smem[];
   float* As = lg_smem;             // [32][LD]
   float* Bs = lg_smem + 32 * LD;   // [64][LD]

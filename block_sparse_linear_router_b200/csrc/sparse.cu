@@ -62,6 +62,8 @@ struct Cfg {
   static_assert(NBAR <= 32, "barrier region");
   static constexpr int OFF_MISC = OFF_BAR + ((8 * NBAR + 15) / 16) * 16;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;         // + alignment slack
+  static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
+  static_assert(!QUANT || 2 * (SMEM + 1024) <= 233472, "two CTAs per SM (228 KB, 1 KB reserved per CTA)");
   static constexpr uint32_t IDESC_QK = QUANT ? make_idesc(2, 1, 1, 128, 64) : make_idesc(1, 1, 1, 128, 64);
   static constexpr uint32_t IDESC_PV = QUANT ? make_idesc(1, 0, 0, 128, D) : make_idesc(1, 1, 1, 128, D);
   static constexpr uint32_t TMEM_COLS = 256;
