@@ -133,3 +133,32 @@ def test_first_heads_projection_everywhere_is_caught(monkeypatch):
         return orig(Q, K, first["w"][0], first["w"][1], smooth)
     monkeypatch.setattr(O, "router_scores", wrong)
     assert _fails(pins.test_router_uses_each_batch_and_heads_own_inputs)
+
+
+def _quantize_q_in_groups(rows_per_group):
+    """Q-hat with the scale taken over groups of `rows_per_group` rows (None:
+    the whole tensor); each 128-row block reports the scale of the group
+    holding its first row."""
+    def wrong(Q):
+        N, d = Q.shape
+        Q32 = np.asarray(Q, dtype=np.float32)
+        g = rows_per_group or N
+        qh = np.zeros((N, d), np.int8)
+        scale_of_row = np.zeros(N, np.float32)
+        for r0 in range(0, N, g):
+            qh[r0:r0 + g], s = O.quant_int8(Q32[r0:r0 + g])
+            scale_of_row[r0:r0 + g] = s
+        return qh, scale_of_row[::O.BQ].copy()
+    return wrong
+
+
+def test_query_quantised_per_64_rows_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "quantize_q", _quantize_q_in_groups(64))
+    assert _fails(pins.test_quantize_q_exact_on_scaled_integer_blocks)
+    assert _fails(pins.test_quantize_q_half_step_per_128_row_block)
+
+
+def test_query_quantised_per_tensor_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "quantize_q", _quantize_q_in_groups(None))
+    assert _fails(pins.test_quantize_q_exact_on_scaled_integer_blocks)
+    assert _fails(pins.test_quantize_q_half_step_per_128_row_block)

@@ -116,6 +116,57 @@ def test_v_quantiser_per_channel_and_zero_channel():
         assert np.all(np.abs(deq - V[:, e]) <= np.abs(V[:, e]) * 2 ** -4 + 2 ** -9 * float(sv[e]) + 1e-12)
 
 
+def _scaled_integer_query_blocks():
+    """Query rows whose 128-row blocks are integers times a power of two, so
+    that symmetric INT8 with scale max|block| / 127 is exact: block i holds
+    integers in [-127, 127] times 2^-i, with one +-127 in its SECOND 64-row
+    half only (its first half stays within +-90). A block-wise quantiser
+    must return those integers and the step 2^-i; a quantiser over 64-row
+    groups would stretch the first half to +-127, and one over the whole
+    tensor would use block 0's step everywhere."""
+    rng = np.random.default_rng(17)
+    nq, d = 4, 32
+    ints = np.zeros((nq * O.BQ, d), np.int64)
+    steps = np.zeros(nq)
+    for i in range(nq):
+        blk = rng.integers(-127, 128, (O.BQ, d))
+        blk[:64] = rng.integers(-90, 91, (64, d))
+        blk[64 + i, 3 + i] = 127 if i % 2 == 0 else -127
+        ints[i * O.BQ:(i + 1) * O.BQ] = blk
+        steps[i] = 2.0 ** -i
+    Q = (ints * np.repeat(steps, O.BQ)[:, None]).astype(np.float64)
+    return Q, ints, steps
+
+
+def test_quantize_q_exact_on_scaled_integer_blocks():
+    """Q-hat is per 128-token query block ([S] step 2: Q and K quantised to
+    INT8 block-wise, with b_q = 128 the query block of [S] step 1): on blocks
+    that are exact multiples of a power-of-two step with a +-127 entry, the
+    codes are the integers and s_q the step, exactly."""
+    Q, ints, steps = _scaled_integer_query_blocks()
+    qh, sq = O.quantize_q(Q)
+    assert qh.shape == Q.shape and sq.shape == (Q.shape[0] // O.BQ,)
+    np.testing.assert_array_equal(qh.astype(np.int64), ints)
+    np.testing.assert_array_equal(sq.astype(np.float64), steps)
+
+
+def test_quantize_q_half_step_per_128_row_block():
+    """On the seeded query rows (magnitudes varying per 64-token block), every
+    128-row block dequantises with ONE scale to within half a step, and the
+    block's largest code is +-127 (the step is as fine as the block allows)."""
+    inp = make_custom(1, 1, 1024, 64, 0.1, seed=18, offset_var=4.0)
+    Q = _head(inp)[0]
+    Q[:64] *= 0.25                           # first half of block 0 much smaller
+    Q = Q.astype(np.float32).astype(np.float64)
+    qh, sq = O.quantize_q(Q)
+    for i in range(Q.shape[0] // O.BQ):
+        rows = slice(i * O.BQ, (i + 1) * O.BQ)
+        deq = qh[rows].astype(np.float64) * float(sq[i])
+        # half a step, plus the fp32 rounding of x * (127 / amax) (a few units in 2^-23 of 127)
+        assert np.max(np.abs(deq - Q[rows])) <= 0.5 * float(sq[i]) * (1 + 1e-4)
+        assert np.abs(qh[rows].astype(np.int64)).max() == 127
+
+
 # ---------------------------------------------------------------- router
 def test_pooling_and_colmean_bruteforce():
     rng = np.random.default_rng(4)
