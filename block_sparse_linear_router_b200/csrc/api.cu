@@ -48,6 +48,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
   s->nq = d->N / BQ;
   s->nk = d->N / BKB;
   s->k = topk_count(s->nk, frac);
+  s->G = linear_chunks(s->BH, s->nk);
   return SLA2_OK;
 }
 
@@ -66,7 +67,7 @@ Layout make_layout(const Shape& s, int quant) {
     return o;
   };
   const size_t BH = s.BH, N = s.N, d = s.d, nq = s.nq, nk = s.nk, k = s.k;
-  const size_t G = linear_chunks(s.BH, s.nk);
+  const size_t G = s.G;
   L.qbar = take(BH * nq * d * 4);
   L.ksum = take(BH * nk * d * 8);
   L.c64 = take(BH * d * 8);
@@ -213,131 +214,33 @@ cudaError_t aux_stream(AuxStream** out) {
   return cudaSuccess;
 }
 
+// Clears the caller's status word (if any) on the call's stream, so that a code
+// left there by an earlier call is not read as this call's.
+cudaError_t clear_status(const sla2_desc* d, cudaStream_t st) {
+  if (!d->status) return cudaSuccess;
+  return cudaMemsetAsync(d->status, 0, sizeof(unsigned), st);
+}
+
 }  // namespace
 
-extern "C" {
+namespace {
 
-const char* sla2_status_string(sla2_status s) {
-  switch (s) {
-    case SLA2_OK: return "ok";
-    case SLA2_ERR_INVALID_ARG: return "invalid argument";
-    case SLA2_ERR_UNSUPPORTED: return "unsupported shape (N % 128 != 0, d not in {64,128}, or too large)";
-    case SLA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
-    case SLA2_ERR_CUDA: return "CUDA error";
-    case SLA2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
-  }
-  return "unknown status";
-}
-
-int sla2_topk_count(int nk, float topk_frac) { return topk_count(nk, topk_frac); }
-
-size_t sla2_workspace_size(const sla2_desc* desc, float topk_frac) {
-  Shape s;
-  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
-  return make_layout(s, desc->quantize).total;
-}
-
-// Test knob: the budget (ns) of every bounded device wait in later launches;
-// 0 restores the default (declared in include/sla2_test.h).
-void sla2_set_wait_budget_ns(unsigned long long ns) { g_budget_ns = ns ? ns : DEFAULT_BUDGET_NS; }
-
-sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
-                        const float* proj_k, float topk_frac, uint8_t* mask_out, int32_t* idx_out,
-                        float* colmean_out, void* stream) {
-  Shape s;
-  sla2_status r = check_desc(desc, topk_frac, &s);
-  if (r != SLA2_OK) return r;
-  if (!q || !k || !proj_q || !proj_k || !mask_out || !idx_out) return SLA2_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
-  const Layout L = make_layout(s, 0);
-  if (!desc->workspace || desc->workspace_bytes < L.total ||
-      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
-    return SLA2_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  r = run_router(desc, s, L, q, k, nullptr, proj_q, proj_k, mask_out, idx_out, 0, st);
-  if (r != SLA2_OK) return r;
-  if (colmean_out)
-    SLA2_TRY(cudaMemcpyAsync(colmean_out, at<float>(desc, L.c32), (size_t)s.BH * s.d * 4, cudaMemcpyDeviceToDevice, st));
-  return SLA2_OK;
-}
-
-sla2_status sla2_router_soft(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
-                             const float* proj_k, float topk_frac, float tau, float* soft_out, float* lambda_out,
-                             void* stream) {
-  Shape s;
-  sla2_status r = check_desc(desc, topk_frac, &s);
-  if (r != SLA2_OK) return r;
-  if (!q || !k || !proj_q || !proj_k || !soft_out) return SLA2_ERR_INVALID_ARG;
-  if (!(tau > 0.f) || !(tau < INFINITY)) return SLA2_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
-  const Layout L = make_layout(s, 0);
-  if (!desc->workspace || desc->workspace_bytes < L.total ||
-      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
-    return SLA2_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  r = router_head(desc, s, L, q, k, nullptr, 0, st);
-  if (r != SLA2_OK) return r;
-  SLA2_TRY(launch_proj(s, desc->H, at<float>(desc, L.qbar), at<float>(desc, L.kbs), proj_q, proj_k,
-                       at<float>(desc, L.A), at<float>(desc, L.Bk), st));
-  float* scores = desc->dbg_scores ? desc->dbg_scores : at<float>(desc, L.scores);
-  SLA2_TRY(launch_scores(s, at<float>(desc, L.A), at<float>(desc, L.Bk), scores, st));
-  SLA2_TRY(launch_soft_topk(s, scores, tau, soft_out, lambda_out, st));
-  return SLA2_OK;
-}
-
-sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v, const float* colmean,
-                              float* h_out, float* z_out, float* Htot_out, float* Ztot_out, void* stream) {
-  Shape s;
-  sla2_status r = check_desc(desc, 1.f, &s);
-  if (r != SLA2_OK) return r;
-  if (!k || !v || !colmean || !h_out || !z_out || !Htot_out || !Ztot_out) return SLA2_ERR_INVALID_ARG;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(h_out) || !aligned16(Htot_out)) return SLA2_ERR_INVALID_ARG;
-  const Layout L = make_layout(s, 0);
-  if (!desc->workspace || desc->workspace_bytes < L.total ||
-      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
-    return SLA2_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  LinearOut o{};
-  o.h = h_out;
-  o.h_mode = 0;
-  o.z = z_out;
-  o.hpart = at<float>(desc, L.hpart);
-  o.zpart = at<float>(desc, L.zpart);
-  o.quant = 0;
-  o.status = desc->status;
-  o.budget_ns = g_budget_ns;
-  SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
-  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, nullptr, Htot_out, Ztot_out, nullptr, nullptr, st));
-  return SLA2_OK;
-}
-
-sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v, const float* proj_q,
-                         const float* proj_k, const float* alpha, float topk_frac, void* out, void* stream) {
-  Shape s;
-  sla2_status r = check_desc(desc, topk_frac, &s);
-  if (r != SLA2_OK) return r;
-  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !out) return SLA2_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj_q) || !aligned16(proj_k) ||
-      !aligned16(out))
-    return SLA2_ERR_INVALID_ARG;
-  if (out == q || out == k || out == v) return SLA2_ERR_INVALID_ARG;
+// The forward pass for the description `desc` and the shape `s` (checked by the
+// caller): `H` heads per batch index the projections and alpha.
+sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Layout& L, const void* q,
+                         const void* k, const void* v, const float* proj_q, const float* proj_k,
+                         const float* alpha, void* out, cudaStream_t st) {
   const int quant = desc->quantize;
-  const Layout L = make_layout(s, quant);
-  if (!desc->workspace || desc->workspace_bytes < L.total ||
-      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
-    return SLA2_ERR_WORKSPACE;
   if (!get_encode()) return SLA2_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t {
     if (!desc->stage_events) return cudaSuccess;
     return cudaEventRecord(static_cast<cudaEvent_t>(desc->stage_events[i]), st);
   };
-  if (desc->status) SLA2_TRY(cudaMemsetAsync(desc->status, 0, sizeof(unsigned), st));
   SLA2_TRY(mark(0));
 
   uint8_t* mask = at<uint8_t>(desc, L.mask);
   int32_t* idx = at<int32_t>(desc, L.idx);
-  r = router_head(desc, s, L, q, k, v, quant, st);
+  sla2_status r = router_head(desc, s, L, q, k, v, quant, st);
   if (r != SLA2_OK) return r;
   SLA2_TRY(mark(1));
 
@@ -412,7 +315,7 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   ea.idx = idx;
   ea.os = os;
   ea.alpha = alpha;
-  ea.H = desc->H;
+  ea.H = H;
   ea.out = out;
   ea.out_f32 = desc->out_dtype;
   ea.ol_dbg = desc->dbg_ol;
@@ -437,6 +340,175 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
     SLA2_TRY(cp(desc->dbg_qscale, L.sq, BH * s.nq * 4));
     SLA2_TRY(cp(desc->dbg_kscale, L.sk, BH * s.nk * 4));
     SLA2_TRY(cp(desc->dbg_vscale, L.sv, BH * s.d * 4));
+  }
+  return SLA2_OK;
+}
+
+}  // namespace
+
+unsigned long long sla2::wait_budget_ns() { return g_budget_ns; }
+
+extern "C" {
+
+const char* sla2_status_string(sla2_status s) {
+  switch (s) {
+    case SLA2_OK: return "ok";
+    case SLA2_ERR_INVALID_ARG: return "invalid argument";
+    case SLA2_ERR_UNSUPPORTED: return "unsupported shape (N % 128 != 0, d not in {64,128}, or too large)";
+    case SLA2_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SLA2_ERR_CUDA: return "CUDA error";
+    case SLA2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+  }
+  return "unknown status";
+}
+
+int sla2_topk_count(int nk, float topk_frac) { return topk_count(nk, topk_frac); }
+
+size_t sla2_workspace_size(const sla2_desc* desc, float topk_frac) {
+  Shape s;
+  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
+  return make_layout(s, desc->quantize).total;
+}
+
+// Test knob: the budget (ns) of every bounded device wait in later launches;
+// 0 restores the default (declared in include/sla2_test.h).
+void sla2_set_wait_budget_ns(unsigned long long ns) { g_budget_ns = ns ? ns : DEFAULT_BUDGET_NS; }
+
+sla2_status sla2_router(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
+                        const float* proj_k, float topk_frac, uint8_t* mask_out, int32_t* idx_out,
+                        float* colmean_out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !proj_q || !proj_k || !mask_out || !idx_out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  r = run_router(desc, s, L, q, k, nullptr, proj_q, proj_k, mask_out, idx_out, 0, st);
+  if (r != SLA2_OK) return r;
+  if (colmean_out)
+    SLA2_TRY(cudaMemcpyAsync(colmean_out, at<float>(desc, L.c32), (size_t)s.BH * s.d * 4, cudaMemcpyDeviceToDevice, st));
+  return SLA2_OK;
+}
+
+sla2_status sla2_router_soft(const sla2_desc* desc, const void* q, const void* k, const float* proj_q,
+                             const float* proj_k, float topk_frac, float tau, float* soft_out, float* lambda_out,
+                             void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !proj_q || !proj_k || !soft_out) return SLA2_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !(tau < INFINITY)) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj_q) || !aligned16(proj_k)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  r = router_head(desc, s, L, q, k, nullptr, 0, st);
+  if (r != SLA2_OK) return r;
+  SLA2_TRY(launch_proj(s, desc->H, at<float>(desc, L.qbar), at<float>(desc, L.kbs), proj_q, proj_k,
+                       at<float>(desc, L.A), at<float>(desc, L.Bk), st));
+  float* scores = desc->dbg_scores ? desc->dbg_scores : at<float>(desc, L.scores);
+  SLA2_TRY(launch_scores(s, at<float>(desc, L.A), at<float>(desc, L.Bk), scores, st));
+  SLA2_TRY(launch_soft_topk(s, scores, tau, soft_out, lambda_out, st));
+  return SLA2_OK;
+}
+
+sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* v, const float* colmean,
+                              float* h_out, float* z_out, float* Htot_out, float* Ztot_out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, 1.f, &s);
+  if (r != SLA2_OK) return r;
+  if (!k || !v || !colmean || !h_out || !z_out || !Htot_out || !Ztot_out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(h_out) || !aligned16(Htot_out)) return SLA2_ERR_INVALID_ARG;
+  const Layout L = make_layout(s, 0);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  LinearOut o{};
+  o.h = h_out;
+  o.h_mode = 0;
+  o.z = z_out;
+  o.hpart = at<float>(desc, L.hpart);
+  o.zpart = at<float>(desc, L.zpart);
+  o.quant = 0;
+  o.status = desc->status;
+  o.budget_ns = g_budget_ns;
+  SLA2_TRY(launch_linear_state(s, k, v, colmean, o, st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, nullptr, Htot_out, Ztot_out, nullptr, nullptr, st));
+  return SLA2_OK;
+}
+
+sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v, const float* proj_q,
+                         const float* proj_k, const float* alpha, float topk_frac, void* out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj_q) || !aligned16(proj_k) ||
+      !aligned16(out))
+    return SLA2_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return SLA2_ERR_INVALID_ARG;
+  const int quant = desc->quantize;
+  const Layout L = make_layout(s, quant);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  return forward_body(desc, s, desc->H, L, q, k, v, proj_q, proj_k, alpha, out, st);
+}
+
+size_t sla2_workspace_size_heads(const sla2_desc* desc, int h_count, float topk_frac) {
+  Shape s;
+  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
+  if (h_count < 1 || h_count > desc->H) return 0;
+  s.BH = h_count;   // one batch index at a time; the chunking stays the full problem's
+  return make_layout(s, desc->quantize).total;
+}
+
+sla2_status sla2_forward_heads(const sla2_desc* desc, int h_begin, int h_count, const void* q, const void* k,
+                               const void* v, const float* proj_q, const float* proj_k, const float* alpha,
+                               float topk_frac, void* out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (h_begin < 0 || h_count < 1 || h_begin > desc->H - h_count) return SLA2_ERR_INVALID_ARG;
+  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !out) return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj_q) || !aligned16(proj_k) ||
+      !aligned16(out))
+    return SLA2_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return SLA2_ERR_INVALID_ARG;
+  if (desc->dbg_scores || desc->dbg_os || desc->dbg_ol || desc->dbg_qhat || desc->dbg_khat || desc->dbg_vhat ||
+      desc->dbg_qscale || desc->dbg_kscale || desc->dbg_vscale || desc->dbg_mask || desc->dbg_idx ||
+      desc->stage_events)
+    return SLA2_ERR_INVALID_ARG;
+  Shape sh = s;
+  sh.BH = h_count;   // s.G (from all B x H heads) fixes the linear state's summation order
+  const Layout L = make_layout(sh, desc->quantize);
+  if (!desc->workspace || desc->workspace_bytes < L.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  const size_t nd = (size_t)s.N * s.d, osz = desc->out_dtype ? 4 : 2;
+  const float* pq = proj_q + (size_t)h_begin * s.d * s.d;
+  const float* pk = proj_k + (size_t)h_begin * s.d * s.d;
+  const float* al = alpha + (size_t)h_begin * s.nq;
+  for (int b = 0; b < desc->B; ++b) {
+    // heads [h_begin, h_begin + h_count) of batch index b are contiguous in [B][H][N][d]
+    const size_t e0 = ((size_t)b * desc->H + h_begin) * nd;
+    r = forward_body(desc, sh, h_count, L, static_cast<const uint16_t*>(q) + e0, static_cast<const uint16_t*>(k) + e0,
+                     static_cast<const uint16_t*>(v) + e0, pq, pk, al, static_cast<uint8_t*>(out) + e0 * osz, st);
+    if (r != SLA2_OK) return r;
   }
   return SLA2_OK;
 }

@@ -19,6 +19,7 @@ constexpr int BKB = 64;   // key block (b_k)
 
 struct Shape {
   int BH, N, d, nq, nk, k;
+  int G;   // key-block chunks per head of the linear-state pass (fixes H_total's summation order)
 };
 
 // ---- router (router.cu) ----------------------------------------------------
@@ -29,6 +30,9 @@ cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void
                         int8_t* qhat, float* sq, unsigned* vamax, unsigned* status, unsigned long long budget_ns,
                         cudaStream_t st);
 constexpr unsigned long long kDefaultWaitBudgetNs = 2000000000ull;   // 2 s per device wait
+// The budget every bounded device wait of the next launches gets (the default, or the
+// value last set by sla2_set_wait_budget_ns); implemented in api.cu.
+unsigned long long wait_budget_ns();
 // colmean (fp64 and fp32) from the per-block sums, and the smoothed pooled keys.
 cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, float* kbar_s,
                            cudaStream_t st);
@@ -67,7 +71,8 @@ struct LinearOut {
   unsigned* status;
   unsigned long long budget_ns;
 };
-// number of key-block chunks (CTAs) per head of the linear-state pass
+// number of key-block chunks (CTAs) per head of the linear-state pass for BH heads in
+// one launch; the launch itself uses Shape::G
 int linear_chunks(int BH, int nk);
 cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, const float* c32, const LinearOut& o,
                                 cudaStream_t st);

@@ -534,7 +534,7 @@ cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, co
   const uint64_t rows = (uint64_t)s.BH * s.N;
   if (!make_tmap_2d(&tk, k, 2, s.d, rows, 64, BKB, 128) || !make_tmap_2d(&tv, v, 2, s.d, rows, 64, BKB, 128))
     return cudaErrorInvalidValue;
-  dim3 grid(linear_chunks(s.BH, s.nk), s.BH);
+  dim3 grid(s.G, s.BH);
   if (s.d == 128) {
     auto kern = linear_state_kernel<128>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LinCfg<128>::SMEM);
@@ -551,7 +551,7 @@ cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float
                                  float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st) {
   const int DD = s.d * s.d;
   dim3 grid((DD + 255) / 256, s.BH);
-  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, linear_chunks(s.BH, s.nk), s.d, s.N, vamax, Htot, Ztot,
+  linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, s.G, s.d, s.N, vamax, Htot, Ztot,
                                              htile, hscale);
   return cudaGetLastError();
 }

@@ -107,10 +107,11 @@ extern "C" sla2_status sla2_router_noalloc(const sla2_desc* desc, const void* q,
   if (scratch_address(&base) != cudaSuccess) return SLA2_ERR_CUDA;
   unsigned char* p = static_cast<unsigned char*>(base);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (desc->status && cudaMemsetAsync(desc->status, 0, sizeof(unsigned), st) != cudaSuccess) return SLA2_ERR_CUDA;
   auto f32 = [&](size_t off) { return reinterpret_cast<float*>(p + off); };
   auto f64 = [&](size_t off) { return reinterpret_cast<double*>(p + off); };
-  if (sla2::launch_pool(s, q, k, nullptr, f32(L.qbar), f64(L.ksum), nullptr, nullptr, nullptr, nullptr,
-                        sla2::kDefaultWaitBudgetNs, st) != cudaSuccess)
+  if (sla2::launch_pool(s, q, k, nullptr, f32(L.qbar), f64(L.ksum), nullptr, nullptr, nullptr, desc->status,
+                        sla2::wait_budget_ns(), st) != cudaSuccess)
     return SLA2_ERR_CUDA;
   if (sla2::launch_colmean(s, f64(L.ksum), f64(L.c64), f32(L.c32), f32(L.kbs), st) != cudaSuccess)
     return SLA2_ERR_CUDA;

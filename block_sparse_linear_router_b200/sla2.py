@@ -54,6 +54,9 @@ SIGNATURES = {
     "sla2_linear_state": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 8),
     "sla2_forward": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 6 + [ctypes.c_float]
                      + [ctypes.c_void_p] * 2),
+    "sla2_workspace_size_heads": (ctypes.c_size_t, [ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_float]),
+    "sla2_forward_heads": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 6
+                           + [ctypes.c_float] + [ctypes.c_void_p] * 2),
 }
 
 _lib = None
@@ -245,3 +248,44 @@ def forward(q, k, v, proj_q, proj_k, alpha, frac, quantize=1, out_dtype=torch.bf
     if r != 0:
         raise Sla2Error(r, "sla2_forward")
     return (out, dbg) if debug else out
+
+
+def shard_heads(H: int, world_size: int, rank: int):
+    """Contiguous head range (h_begin, h_count) of `rank` when H heads are split
+    over `world_size` ranks as evenly as possible (the first H % world_size
+    ranks take one head more). A rank may get h_count = 0 when world_size > H."""
+    if world_size < 1 or not (0 <= rank < world_size) or H < 0:
+        raise ValueError("bad head sharding arguments")
+    base, extra = divmod(H, world_size)
+    h_begin = rank * base + min(rank, extra)
+    return h_begin, base + (1 if rank < extra else 0)
+
+
+def workspace_size_heads(B, H, N, d, h_count, frac, quantize=1) -> int:
+    desc = make_desc(B, H, N, d, quantize)
+    return load_library().sla2_workspace_size_heads(ctypes.byref(desc), h_count, frac)
+
+
+def forward_heads(q, k, v, proj_q, proj_k, alpha, frac, h_begin, h_count, out, quantize=1,
+                  workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, stream=None):
+    """Heads [h_begin, h_begin + h_count) of the forward pass, written into the full
+    output tensor `out` [B,H,N,d] (bf16 or fp32); nothing else of `out` is touched.
+    Bit-identical to those heads of forward() on the same full inputs."""
+    lib = load_library()
+    _check_qkv(q, k, v, proj_q, proj_k, alpha, out)
+    B, H, N, d = q.shape
+    if out.dtype not in (torch.bfloat16, torch.float32) or tuple(out.shape) != (B, H, N, d):
+        raise ValueError("out must be a bf16 or fp32 [B,H,N,d] tensor")
+    n = lib.sla2_workspace_size_heads(ctypes.byref(make_desc(B, H, N, d, quantize)), h_count, frac)
+    if n == 0:
+        raise Sla2Error(1, "sla2_workspace_size_heads")
+    ws = workspace if workspace is not None else torch.empty(n, dtype=torch.uint8, device=q.device)
+    desc = make_desc(B, H, N, d, quantize, 1 if out.dtype == torch.float32 else 0)
+    desc.workspace, desc.workspace_bytes = ws.data_ptr(), ws.numel()
+    if status is not None:
+        desc.status = status.data_ptr()
+    r = lib.sla2_forward_heads(ctypes.byref(desc), h_begin, h_count, _ptr(q), _ptr(k), _ptr(v), _ptr(proj_q),
+                               _ptr(proj_k), _ptr(alpha), frac, _ptr(out), _stream(stream))
+    if r != 0:
+        raise Sla2Error(r, "sla2_forward_heads")
+    return out

@@ -33,6 +33,10 @@
  *     may run concurrently need separate workspaces.
  *   - Device-side waits are bounded; a wait that runs out writes a nonzero code
  *     into the optional status word (desc.status) and the kernel returns.
+ *   - The library keeps per-device state for the life of the process (the
+ *     auxiliary stream of sla2_forward, the device address of the fixed array
+ *     of sla2_router_noalloc). Do not keep using the library on a device after
+ *     cudaDeviceReset on it: that state would refer to the destroyed context.
  */
 #ifndef SLA2_H
 #define SLA2_H
@@ -62,9 +66,10 @@ typedef struct {
   void* workspace;     /* device scratch, >= sla2_workspace_size() bytes,
                           256-byte aligned                                      */
   size_t workspace_bytes;
-  unsigned int* status;/* optional device word; set to 0 at each call and to a
-                          nonzero SLA2_ERR_DEVICE_TIMEOUT code if a bounded
-                          device wait ran out                                   */
+  unsigned int* status;/* optional device word; every entry point clears it on
+                          `stream` before its first launch, and a bounded
+                          device wait that runs out sets it to
+                          SLA2_ERR_DEVICE_TIMEOUT                               */
   /* Optional debug exports (NULL = not written), all device pointers:        */
   float* dbg_scores;   /* router logits s, fp32 [B][H][N/128][N/64]            */
   float* dbg_os;       /* sparse branch O_s, fp32 [B][H][N][d]                 */
@@ -140,7 +145,9 @@ sla2_status sla2_router_soft(const sla2_desc* desc, const void* q, const void* k
  *   - Shapes whose router scratch exceeds the array are rejected with
  *     SLA2_ERR_WORKSPACE before anything is launched. The scratch is about
  *     (5/16) N d + N^2 / 2048 bytes per (batch, head): 1.84 MB for N = 32768,
- *     d = 128, so up to 8 such heads fit in one call.
+ *     d = 128, so up to 9 such heads fit in one call.
+ *   - desc->status is honoured as in sla2_router (cleared, then set if a
+ *     bounded device wait runs out), and so is sla2_set_wait_budget_ns.
  *   - The first call on each device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first call
  *     before any stream capture.
@@ -188,6 +195,27 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
 sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v,
                          const float* proj_q, const float* proj_k, const float* alpha,
                          float topk_frac, void* out, void* stream);
+
+/* One rank's share of a head-sharded forward pass (the summary page's
+ * future-work paragraph names multi-GPU execution; every step of the pass is
+ * independent per (batch, head), so a contiguous range of heads per GPU needs
+ * no collective).
+ *   desc  : the FULL problem (B, H, N, d, quantize, out_dtype, workspace, status);
+ *           its debug exports and stage_events must be NULL (else
+ *           SLA2_ERR_INVALID_ARG).
+ *   q, k, v, out : the full [B][H][N][d] tensors; proj_q/proj_k: the full
+ *           [H][d][d]; alpha: the full [H][N/128].
+ *   Computes out[b][h] for every b and every h in [h_begin, h_begin + h_count)
+ *   and writes nothing else of out. Those heads are bit-identical to the ones
+ *   sla2_forward writes for the same full description (the linear state's
+ *   chunking, which fixes its summation order, is taken from all B x H heads).
+ *   Workspace: sla2_workspace_size_heads(desc, h_count, frac) bytes, reused for
+ *   each batch index in turn (one pass of the forward per batch index, in
+ *   order, on `stream`). 0 <= h_begin, 1 <= h_count, h_begin + h_count <= H. */
+size_t sla2_workspace_size_heads(const sla2_desc* desc, int h_count, float topk_frac);
+sla2_status sla2_forward_heads(const sla2_desc* desc, int h_begin, int h_count, const void* q, const void* k,
+                               const void* v, const float* proj_q, const float* proj_k, const float* alpha,
+                               float topk_frac, void* out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -135,3 +135,19 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises((ValueError, RuntimeError)):
         sla2.forward(q, q, q, torch.zeros(1, 64, 64), torch.zeros(1, 64, 64), torch.zeros(1, 1), 0.5)
+
+
+def test_head_range_entry_point_rejects_bad_ranges_on_the_host(lib):
+    buf, p = _fake()
+    ws, pws = _fake()
+    d = _desc(H=4)
+    n = lib.sla2_workspace_size_heads(ctypes.byref(d), 2, 0.1)
+    assert 0 < n < lib.sla2_workspace_size(ctypes.byref(d), 0.1)
+    for hc in (0, -1, 5):
+        assert lib.sla2_workspace_size_heads(ctypes.byref(d), hc, 0.1) == 0
+    d.workspace, d.workspace_bytes = pws, 1 << 20
+    args = [ctypes.c_void_p(p)] * 6 + [ctypes.c_float(0.1), ctypes.c_void_p(p + 4096), None]
+    for hb, hc in ((-1, 2), (3, 2), (0, 0), (4, 1)):
+        assert lib.sla2_forward_heads(ctypes.byref(d), hb, hc, *args) == 1      # invalid argument
+    d.dbg_scores = p                                                             # debug exports refused
+    assert lib.sla2_forward_heads(ctypes.byref(d), 0, 2, *args) == 1
