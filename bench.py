@@ -45,6 +45,44 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+def measure_8bit_peaks(device, n=8192, reps=10):
+    """Dense 8-bit tensor-core peaks of this GPU, measured live with the library
+    GEMMs PyTorch ships (cuBLASLt): torch._int_mm (int8 x int8 -> int32) and
+    torch._scaled_mm (e4m3 x e4m3 -> bf16) at n^3, best of `reps` after warm-up,
+    CUDA events on the current stream (burst figures). Returns {"int8": TOPS,
+    "e4m3": TOPS} with None for a GEMM that is unavailable."""
+    import torch
+    out = {}
+    a8 = torch.randint(-64, 64, (n, n), dtype=torch.int8, device=device)
+    b8 = torch.randint(-64, 64, (n, n), dtype=torch.int8, device=device).t()   # column-major B
+    af = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+    bf = torch.randn(n, n, device=device).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), dtype=torch.float32, device=device)
+    fns = {"int8": lambda: torch._int_mm(a8, b8),
+           "e4m3": lambda: torch._scaled_mm(af, bf, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)}
+    for name, fn in fns.items():
+        try:
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize(device)
+            best = float("inf")
+            for _ in range(reps):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize(device)
+                best = min(best, e0.elapsed_time(e1))
+            out[name] = 2.0 * n ** 3 / (best * 1e-3) / 1e12
+        except Exception as exc:   # a GEMM this torch build cannot run here
+            out[name] = None
+            out[name + "_error"] = f"{type(exc).__name__}: {exc}"[:200]
+    del a8, b8, af, bf
+    torch.cuda.empty_cache()
+    return out
+
+
 def work_model(w, k):
     """Algorithmic work of one forward pass: bytes of the HBM-bound stages, 8-bit ops
     of the sparse branch and fp16 flops of the epilogue, per the definitions below."""
@@ -55,6 +93,9 @@ def work_model(w, k):
     return {
         "pairs": pairs,
         "sparse_ops": pairs * 4 * 128 * 64 * d,
+        # half of them INT8 (Q-hat K-hat^T), half e4m3 (P-hat V-hat)
+        "sparse_ops_i8": pairs * 2 * 128 * 64 * d,
+        "sparse_ops_f8": pairs * 2 * 128 * 64 * d,
         "effective_ops": 4 * B * H * N * N * d,
         # router: read Q, K, V (bf16), write Q-hat (int8)
         "router_bytes": 2 * E * 3 + E,
@@ -64,8 +105,10 @@ def work_model(w, k):
         # repeated tile gather (k + 1 per query block) is L2 traffic, reported separately
         "epilogue_bytes": 2 * E + 4 * E + 2 * E + BH * nk * d * d * 2,
         "gather_bytes": BH * nq * (k + 1) * d * d * 2,   # per query block: H_total and the k selected h_j tiles
-        # epilogue MMAs: phi(Q_i) (128 x d) times k + 1 tiles (d x d), fp16 in, fp32 accumulate
-        "epilogue_flops": BH * nq * (k + 1) * 2 * 128 * d * d if k < nk else 0,
+        # epilogue MMAs as issued: phi(Q_i) (128 x d) times k + 1 tiles (d x d), fp16 in, fp32
+        # accumulate; the algorithmic work is one product phi(Q_i) H_i per query block
+        "epilogue_flops_issued": BH * nq * (k + 1) * 2 * 128 * d * d if k < nk else 0,
+        "epilogue_flops": 2 * N * d * d * BH if k < nk else 0,
     }
 
 
@@ -195,39 +238,73 @@ def dist_setup():
     return ws, rank, local
 
 
-def cpu_oracle_sample(w, blocks_per_head=16):
-    """Time the oracle on a bounded sample of the workload: one head's set-up
-    (router, quantisation, linear states) plus `blocks_per_head` query blocks,
-    extrapolated to the whole workload. Returns (effective TOPS, description)."""
-    import numpy as np
+def _oracle_head_task(args):
+    """One head of the oracle (mode qa) on the bounded sample, single-threaded:
+    its set-up (router, quantisation, linear states), then the set-up again with
+    the first `nb` query blocks. Returns (set-up s, query-block s)."""
+    Q, K, V, Wq, Wk, al, frac, nb = args
+    from threadpoolctl import threadpool_limits
     from oracle import sla2_oracle as O
-    from block_sparse_linear_router_b200.inputs import make_inputs
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    inp = make_inputs(w, heads=1)
-    Q, K, V = (t[0, 0].double().numpy() for t in (inp.q, inp.k, inp.v))
-    Wq, Wk, al = inp.proj_q[0].double().numpy(), inp.proj_k[0].double().numpy(), inp.alpha[0].double().numpy()
-    t0 = time.perf_counter()
-    O.head_forward(Q, K, V, Wq, Wk, al, w.topk_frac, mode="qa", blocks=[])
-    t_setup = time.perf_counter() - t0
-    nb = blocks_per_head
-    t0 = time.perf_counter()
-    O.head_forward(Q, K, V, Wq, Wk, al, w.topk_frac, mode="qa", blocks=list(range(nb)))
-    t_blocks = max(time.perf_counter() - t0 - t_setup, 1e-9)
-    per_block = t_blocks / nb
-    nq = w.N // 128
-    t_full = w.B * w.H * (t_setup + nq * per_block)
-    eff = 4 * w.B * w.H * w.N * w.N * w.d / t_full / 1e12
-    sample = (f"oracle mode qa, 1 head: set-up {t_setup:.2f} s + {nb} query blocks {t_blocks:.2f} s, "
-              f"extrapolated to {w.B * w.H} heads x {nq} query blocks = {t_full:.0f} s per forward")
-    return eff, sample, cores, t_full
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        O.head_forward(Q, K, V, Wq, Wk, al, frac, mode="qa", blocks=[])
+        t1 = time.perf_counter()
+        O.head_forward(Q, K, V, Wq, Wk, al, frac, mode="qa", blocks=list(range(nb)))
+        t2 = time.perf_counter()
+    setup = t1 - t0
+    return setup, max((t2 - t1) - setup, 1e-9)
+
+
+class OracleSampler:
+    """The CPU oracle timed on the host cores: one single-threaded worker process
+    per core (spawned, so it is safe after CUDA has been initialised), each head of
+    the workload one task (its set-up plus its first `nb` query blocks). The full
+    forward time is extrapolated from the per-head times: every head's set-up plus
+    nq / nb times its query-block time, the heads spread over the workers."""
+
+    def __init__(self, w, nb):
+        import multiprocessing as mp
+        from block_sparse_linear_router_b200.inputs import make_inputs
+        self.w, self.nb = w, nb
+        inp = make_inputs(w)
+        self.tasks = []
+        for b in range(w.B):
+            for h in range(w.H):
+                f = lambda t: t[b, h].float().numpy()       # bf16 values, exact in fp32
+                self.tasks.append((f(inp.q), f(inp.k), f(inp.v), inp.proj_q[h].double().numpy(),
+                                   inp.proj_k[h].double().numpy(), inp.alpha[h].double().numpy(),
+                                   w.topk_frac, nb))
+        self.cores = max(1, min(len(self.tasks), os.cpu_count() or 1))
+        self.pool = mp.get_context("spawn").Pool(self.cores)
+
+    def step(self):
+        """One bounded sample: (wall s, extrapolated full-forward s, description)."""
+        import math
+        w, nb = self.w, self.nb
+        t0 = time.perf_counter()
+        res = self.pool.map(_oracle_head_task, self.tasks, chunksize=1)
+        wall = time.perf_counter() - t0
+        nq = w.N // 128
+        per_head = sorted((su + nq / nb * bl for su, bl in res), reverse=True)
+        rounds = math.ceil(len(per_head) / self.cores)
+        t_full = sum(per_head) / self.cores if rounds > 1 else per_head[0]
+        su = statistics.mean(r[0] for r in res)
+        bl = statistics.mean(r[1] for r in res)
+        desc = (f"oracle mode qa, {len(res)} heads on {self.cores} single-threaded worker processes: per head "
+                f"set-up {su:.2f} s + {nb} of {nq} query blocks {bl:.2f} s (sample wall {wall:.1f} s); "
+                f"extrapolated full forward {t_full:.3g} s")
+        return wall, t_full, desc
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle, rank 0 only."""
+    """--impl reference: the CPU oracle on the host cores, rank 0 only. Each step is
+    one bounded sample of the workload (every head's set-up and its first 8 query
+    blocks); `ms_per_step` is that sample's measured wall time and `value` the
+    effective TOPS of the full forward extrapolated from it."""
     from block_sparse_linear_router_b200.inputs import WORKLOADS
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -237,20 +314,27 @@ def run_reference(args):
     if args.frac is not None:
         w = w.with_frac(args.frac, alpha_one=(args.frac == 1.0))
     k = O.topk_count(w.nk, w.topk_frac)
-    vals, samples = [], []
-    for _ in range(max(args.warmup, 0)):
-        cpu_oracle_sample(w, blocks_per_head=8)
-    for _ in range(args.steps):
-        eff, sample, cores, t_full = cpu_oracle_sample(w, blocks_per_head=8)
-        vals.append(eff)
-        samples.append(sample)
-    v = statistics.median(vals)
+    sampler = OracleSampler(w, nb=8)
+    try:
+        for _ in range(max(args.warmup, 0)):
+            sampler.step()
+        walls, fulls, desc = [], [], ""
+        for _ in range(args.steps):
+            wall, t_full, desc = sampler.step()
+            walls.append(wall)
+            fulls.append(t_full)
+    finally:
+        sampler.close()
+    t_full = statistics.median(fulls)
+    v = 4 * w.B * w.H * w.N * w.N * w.d / t_full / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 4 * w.B * w.H * w.N * w.N * w.d / v / 1e9,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(walls) * 1e3,
+        "ms_per_step_is": "measured wall time of one bounded sample (value is extrapolated to the full forward)",
+        "extrapolated_forward_ms": t_full * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": bench_config(w, k, args.gpus),
-        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": samples[-1]},
+        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": sampler.cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -267,6 +351,7 @@ def main():
     ap.add_argument("--frac", type=float, default=None, help="override k% (sweep)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-peaks", action="store_true", help="skip the live 8-bit GEMM peak measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -384,26 +469,42 @@ def main():
 
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
-    p8 = peaks["bf16_tflops"] * NOMINAL_8BIT_OVER_BF16
+    p16 = peaks["bf16_tflops"]   # fp16 and bf16 run at the same dense rate
+    # 8-bit peak of the sparse branch: its INT8 half at the measured int8 rate and its
+    # e4m3 half at the measured e4m3 rate (t_min = ops_i8 / P_i8 + ops_f8 / P_f8);
+    # without a measurement, the bf16 figure times the nominal 8-bit : bf16 ratio
+    p8_meas = measure_8bit_peaks(dev) if not args.no_peaks else {}
+    if p8_meas.get("int8") and p8_meas.get("e4m3"):
+        t_min = wm["sparse_ops_i8"] / p8_meas["int8"] + wm["sparse_ops_f8"] / p8_meas["e4m3"]
+        p8 = wm["sparse_ops"] / t_min
+        p8_src = (f"measured int8/fp8 (torch._int_mm {p8_meas['int8']:.0f} TOPS, torch._scaled_mm e4m3 "
+                  f"{p8_meas['e4m3']:.0f} TOPS, 8192^3 burst, this run)")
+    else:
+        p8 = p16 * NOMINAL_8BIT_OVER_BF16
+        p8_src = f"{peak_src} bf16 burst x 2 (nominal 8-bit : bf16 ratio; 8-bit GEMMs not measured)"
     names = ["router", "linear_state", "sparse", "epilogue"]
     kern = {}
-    p16 = peaks["bf16_tflops"]   # fp16 and bf16 run at the same dense rate
     for n, msv in zip(names, stage_ms):
         if n == "sparse":
             ach = wm["sparse_ops"] / (msv * 1e-3) / 1e12
-            kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p8, "unit": "TOPS", "frac": ach / p8}
-        elif n == "epilogue" and wm["epilogue_flops"] > 0:
-            # tensor-bound when its MMA time exceeds its HBM time (206 GFLOP vs 604 MB here)
-            ach = wm["epilogue_flops"] / (msv * 1e-3) / 1e12
-            hb = wm["epilogue_bytes"] / (msv * 1e-3) / 1e9
-            kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p16, "unit": "TFLOP/s",
-                       "frac": ach / p16, "hbm_achieved_gbs": hb, "hbm_frac": hb / hbm,
-                       "algorithmic_bytes": wm["epilogue_bytes"], "flops": wm["epilogue_flops"]}
-        else:
-            b = wm[f"{n.split('_')[0]}_bytes"] if n != "linear_state" else wm["linear_bytes"]
+            kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p8, "unit": "TOPS", "frac": ach / p8,
+                       "peak_source": p8_src}
+        elif n == "epilogue":
+            # HBM-bound: read Q (bf16) and O_s (fp32), the h tiles once, write out; its
+            # tensor work is given beside it (algorithmic: one phi(Q_i) H_i per query block)
+            b = wm["epilogue_bytes"]
             ach = b / (msv * 1e-3) / 1e9
             kern[n] = {"ms": msv, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                       "algorithmic_bytes": b}
+                       "algorithmic_bytes": b, "peak_source": f"{peak_src} HBM copy",
+                       "tensor_algorithmic_flops": wm["epilogue_flops"],
+                       "tensor_issued_flops": wm["epilogue_flops_issued"],
+                       "tensor_frac_algorithmic": wm["epilogue_flops"] / (msv * 1e-3) / 1e12 / p16,
+                       "tensor_frac_issued": wm["epilogue_flops_issued"] / (msv * 1e-3) / 1e12 / p16}
+        else:
+            b = wm["router_bytes"] if n == "router" else wm["linear_bytes"]
+            ach = b / (msv * 1e-3) / 1e9
+            kern[n] = {"ms": msv, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                       "algorithmic_bytes": b, "peak_source": f"{peak_src} HBM copy"}
     for n in names:
         tb, tsrc = measured_traffic(n)
         kern[n]["traffic"] = tb
@@ -411,15 +512,18 @@ def main():
             kern[n]["traffic_source"] = tsrc
     dom = max(names, key=lambda n: kern[n]["ms"])
     dk = kern[dom]
-    psrc = {"sparse": "8-bit = bf16 burst x 2 nominal ratio", "epilogue": "fp16 = bf16 burst (same dense rate)"}
     roofline = {"bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"], "unit": dk["unit"],
-                "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dom,
-                "peak_source": f"{peak_src} ({psrc.get(dom, 'HBM copy') if dk['bound'] == 'tensor' else 'HBM copy'})"}
+                "frac": dk["frac"], "traffic": dk["traffic"], "kernel": dom, "peak_source": dk["peak_source"]}
 
     cpu = None
-    if not args.no_cpu_baseline:
-        eff, sample, cores, _ = cpu_oracle_sample(w)
-        cpu = {"value": eff, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample}
+    if not args.no_cpu_baseline and ws == 1:
+        sampler = OracleSampler(w, nb=16)
+        try:
+            _, t_full, sample = sampler.step()
+        finally:
+            sampler.close()
+        cpu = {"value": wm["effective_ops"] / t_full / 1e12, "unit": "TOPS", "cores": sampler.cores,
+               "kind": "oracle", "sample": sample}
 
     line = {
         "metric": METRIC, "value": eff_tops, "unit": "TOPS", "n_gpus": ws, "steps": K, "warmup": args.warmup,
@@ -433,6 +537,7 @@ def main():
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_forward(w, k) * K, "clocks": clk,
         "sparse_issued_tops": kern["sparse"]["achieved"],
+        "peaks_8bit_tops": p8_meas or None,
     }
     print(json.dumps(line), flush=True)
     if ws > 1:
