@@ -336,6 +336,18 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Register reallocation for a warpgroup (all four of its warps execute it):
+// release registers down to N a thread, or wait for the CTA's released
+// registers to raise this warpgroup to N a thread.
+template <int N>
+__device__ __forceinline__ void regs_release() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_claim() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes' worth)
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -360,6 +372,32 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// 2^t for two fp32 values at once on the FMA pipe (no MUFU), for t <= 2^22:
+// Cody-Waite style range reduction t = j + f with j = rint(t) and f in
+// [-1/2, 1/2] (the rounding by the 1.5 * 2^23 add), a cubic minimax
+// polynomial for 2^f (coefficients fitted here by the Remez exchange on
+// relative error over [-1/2, 1/2]: max relative error 7.5e-5 in exact
+// arithmetic), and the scaling by 2^j as an integer add to the exponent
+// field. t is clamped below at -125 so that 2^j stays a normal number; the
+// results there (about 2^-125) are below every use of them.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
+  float t0, t1;
+  f2_unpack(t2, t0, t1);
+  t2 = f2_pack(fmaxf(t0, -125.f), fmaxf(t1, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f), neg_magic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t r = f2_add(t2, magic);                                        // 1.5 * 2^23 + j
+  const uint64_t f = f2_fma(f2_add(r, neg_magic), f2_pack(-1.f, -1.f), t2);    // t - j, exact
+  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f, f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float r0, r1, p0, p1;
+  f2_unpack(r, r0, r1);
+  f2_unpack(p, p0, p1);
+  // the low bits of r hold j; shifted by 23 they add j to p's exponent
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
