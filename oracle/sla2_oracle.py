@@ -41,6 +41,17 @@ Modes of ``forward``:
   "qa" quantised, online softmax in the tile order above (the contract);
   "qb" quantised, with each row's exact final max (schedule-free bound);
   "u"  unquantised, exact masked softmax attention.
+
+Backward pass (``head_backward``): the gradient of the unquantised forward
+with respect to Q, K, V and alpha for a given block mask ([D] §7 note 3: a
+hand-derived gradient, in which the linear branch's dH_i and dZ_i are formed
+once per query block; [D] §2 table: the low-bit kernels are forward-only and
+the backward runs in 16-bit, so the gradient is that of the unquantised
+pass). Readings: the hard Top-k mask is piecewise constant in Q, K and the
+projections, so it is held fixed and the router's projections receive no
+gradient from this path (in training the pages route the gradient through
+SoftTop-k, which is a separate function here); K smoothing is part of the
+differentiated map.
 """
 from __future__ import annotations
 
@@ -430,3 +441,131 @@ def router(q, k, proj_q, proj_k, frac):
             scores[b, hh] = s
             masks[b, hh], idxs[b, hh] = topk_mask(s, kk)
     return masks, idxs, scores
+
+
+# --------------------------------------------------------------------------
+# Backward pass of the unquantised forward for a fixed mask ([D] §7 note 3)
+# --------------------------------------------------------------------------
+def feature_softmax_backward(Y, dY) -> np.ndarray:
+    """Gradient through phi = softmax over the features: given Y = phi(X) and
+    dY = dL/dY (rows), returns dL/dX = Y * (dY - rowsum(dY * Y))."""
+    Y = np.asarray(Y, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    return Y * (dY - np.sum(dY * Y, axis=-1, keepdims=True))
+
+
+def head_forward_masked(Q, K, V, alpha_h, mask):
+    """Unquantised forward of one head for a GIVEN block mask (the function the
+    backward differentiates): O = alpha O_s + (1 - alpha) O_l with O_s the
+    softmax attention over the selected keys ([S] step 2) and O_l the linear
+    attention over the unselected key blocks ([S] step 3), K smoothed first
+    ([D] §7 note 1). Returns O [N, d]."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    N, d = Q.shape
+    Ks = K - colmean(K)
+    h, z = linear_states(Ks, V)
+    O = np.zeros((N, d))
+    for i in range(N // BQ):
+        sel = np.nonzero(mask[i])[0]
+        rows = slice(i * BQ, (i + 1) * BQ)
+        os_i = sparse_exact(Q, Ks, V, sel, i, d) if len(sel) else np.zeros((BQ, d))
+        ol_i = linear_branch(Q, h, z, mask[i], i)
+        a = float(alpha_h[i])
+        O[rows] = a * os_i + (1.0 - a) * ol_i
+    return O
+
+
+def unselected_blocks(mask_row) -> np.ndarray:
+    """Key blocks of one mask row whose states h_j, z_j enter H_i, Z_i (the
+    unselected ones, [S] step 3)."""
+    return np.nonzero(np.asarray(mask_row) == 0)[0]
+
+
+def head_backward(Q, K, V, alpha_h, mask, dO):
+    """dL/dQ, dL/dK, dL/dV [N, d] and dL/dalpha [nq] of one head, for the
+    upstream gradient dO = dL/dO, by the chain rule through the unquantised
+    forward with the mask held fixed. Per query block i (rows r of block i):
+
+      sparse branch (softmax over the selected keys, S = Q_i K_s^T / sqrt(d)):
+        dV_sel += P^T dO_s,  dP = dO_s V_sel^T,  dS = P * (dP - rowsum(dP * P)),
+        dQ_i += dS K_sel / sqrt(d),  dK_sel += dS^T Q_i / sqrt(d);
+      linear branch (a = phi(Q_i), num = a H_i, den = a Z_i, O_l = num / den):
+        dnum = dO_l / den,  dden = -rowsum(dO_l * O_l) / den,
+        da = dnum H_i^T + dden Z_i^T,  dQ_i += phi-backward(a, da),
+        dH_i = a^T dnum,  dZ_i = a^T dden  (formed once per query block);
+      mix: dO_s = alpha_i dO, dO_l = (1 - alpha_i) dO,
+        dalpha_i = sum over the block's rows and channels of dO * (O_s - O_l).
+
+    Then, per key block j, the plain definition dh_j = sum of dH_i and
+    dz_j = sum of dZ_i over the query blocks i that did NOT select j (h_j, z_j
+    enter exactly those H_i, Z_i), and through h_j = phi(K_j)^T V_j,
+    z_j = phi(K_j)^T 1: dV_j += phi(K_j) dh_j, dphi(K_j) = V_j dh_j^T + dz_j,
+    dK_s += phi-backward(phi(K_j), dphi(K_j)). Finally through K_s = K - colmean(K):
+    dK = dK_s - colmean(dK_s)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    N, d = Q.shape
+    nq, nk = N // BQ, N // BK
+    Ks = K - colmean(K)
+    h, z = linear_states(Ks, V)
+    rs = 1.0 / math.sqrt(d)
+    dQ = np.zeros((N, d))
+    dKs = np.zeros((N, d))
+    dV = np.zeros((N, d))
+    dalpha = np.zeros(nq)
+    dh = np.zeros((nk, d, d))
+    dz = np.zeros((nk, d))
+    for i in range(nq):
+        rows = slice(i * BQ, (i + 1) * BQ)
+        sel = np.nonzero(mask[i])[0]
+        unsel = unselected_blocks(mask[i])
+        al = float(alpha_h[i])
+        dOs = al * dO[rows]
+        dOl = (1.0 - al) * dO[rows]
+        Qi = Q[rows]
+        # sparse branch
+        if len(sel):
+            keys = np.concatenate([np.arange(j * BK, (j + 1) * BK) for j in sel])
+            S = (Qi @ Ks[keys].T) * rs
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            Os = P @ V[keys]
+            dV[keys] += P.T @ dOs
+            dP = dOs @ V[keys].T
+            dS = P * (dP - np.sum(dP * P, axis=1, keepdims=True))
+            dQ[rows] += (dS @ Ks[keys]) * rs
+            dKs[keys] += (dS.T @ Qi) * rs
+        else:
+            Os = np.zeros((BQ, d))
+        # linear branch
+        if len(unsel):
+            Hi = h[unsel].sum(axis=0)
+            Zi = z[unsel].sum(axis=0)
+            a = feature_softmax(Qi)
+            num = a @ Hi
+            den = a @ Zi
+            Ol = num / den[:, None]
+            dnum = dOl / den[:, None]
+            dden = -np.sum(dOl * Ol, axis=1) / den
+            da = dnum @ Hi.T + dden[:, None] * Zi[None, :]
+            dQ[rows] += feature_softmax_backward(a, da)
+            dHi = a.T @ dnum
+            dZi = a.T @ dden
+            for j in unsel:
+                dh[j] += dHi
+                dz[j] += dZi
+        else:
+            Ol = np.zeros((BQ, d))
+        dalpha[i] = float(np.sum(dO[rows] * (Os - Ol)))
+    phk = feature_softmax(Ks)
+    for j in range(nk):
+        t = slice(j * BK, (j + 1) * BK)
+        dV[t] += phk[t] @ dh[j]
+        dphi = V[t] @ dh[j].T + dz[j][None, :]
+        dKs[t] += feature_softmax_backward(phk[t], dphi)
+    dK = dKs - dKs.mean(axis=0, keepdims=True)
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dalpha": dalpha}
