@@ -71,6 +71,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 // gets SLA2_DEV_TIMEOUT and the abort flag is raised).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status, uint64_t budget_ns) {
+  // a completed phase is seen by the non-suspending test (cheaper than try_wait)
+  if (mbar_test(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -301,6 +303,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 #undef SLA2_W8
+// The same 32-bit value into 32 consecutive columns of this thread's lane.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -372,14 +382,15 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-// 2^t for two fp32 values at once on the FMA pipe (no MUFU), for t <= 2^22:
+// 2^t for two fp32 values at once on the FMA pipe (no MUFU), for t < 128:
 // Cody-Waite style range reduction t = j + f with j = rint(t) and f in
-// [-1/2, 1/2] (the rounding by the 1.5 * 2^23 add), a cubic minimax
+// [-1/2, 1/2] (the rounding by the 1.5 * 2^23 add), a quartic minimax
 // polynomial for 2^f (coefficients fitted here by the Remez exchange on
-// relative error over [-1/2, 1/2]: max relative error 7.5e-5 in exact
-// arithmetic), and the scaling by 2^j as an integer add to the exponent
-// field. t is clamped below at -125 so that 2^j stays a normal number; the
-// results there (about 2^-125) are below every use of them.
+// relative error over [-1/2, 1/2]: max relative error 2.7e-6 with the
+// coefficients rounded to fp32, 2.9e-6 with fp32 Horner steps), and the
+// scaling by 2^j as an integer add to the exponent field. t is clamped below
+// at -125 so that 2^j stays a normal number; the results there (about
+// 2^-125) are below every use of them.
 __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
   float t0, t1;
   f2_unpack(t2, t0, t1);
@@ -387,9 +398,11 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
   const uint64_t magic = f2_pack(12582912.f, 12582912.f), neg_magic = f2_pack(-12582912.f, -12582912.f);
   const uint64_t r = f2_add(t2, magic);                                        // 1.5 * 2^23 + j
   const uint64_t f = f2_fma(f2_add(r, neg_magic), f2_pack(-1.f, -1.f), t2);    // t - j, exact
-  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f, f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  uint64_t p = f2_fma(f2_pack(0.009570102207362652f, 0.009570102207362652f), f,
+                      f2_pack(0.05591785907745361f, 0.05591785907745361f));
+  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
+  p = f2_fma(p, f, f2_pack(0.6931217908859253f, 0.6931217908859253f));
+  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
   float r0, r1, p0, p1;
   f2_unpack(r, r0, r1);
   f2_unpack(p, p0, p1);
