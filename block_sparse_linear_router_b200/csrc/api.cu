@@ -541,26 +541,3 @@ extern "C" sla2_status sla2_selftest_timeout(unsigned* status, unsigned long lon
   timeout_probe_kernel<<<1, 32, 0, st>>>(status, budget_ns);
   return cuda_status(cudaGetLastError());
 }
-
-// ---------------------------------------------------------------------------
-// Test hook (declared in include/sla2_test.h): the FMA-pipe 2^x of the sparse
-// branch's softmax, elementwise over n fp32 values.
-namespace {
-__global__ void exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float x1 = i + 1 < n ? x[i + 1] : 0.f;
-  float y0, y1;
-  sla2::f2_unpack(sla2::exp2_poly_x2(sla2::f2_pack(x[i], x1)), y0, y1);
-  y[i] = y0;
-  if (i + 1 < n) y[i + 1] = y1;
-}
-}  // namespace
-
-extern "C" sla2_status sla2_selftest_exp2(const float* x, float* y, int n, void* stream) {
-  if (!x || !y || n < 0 || !aligned16(x) || !aligned16(y)) return SLA2_ERR_INVALID_ARG;
-  if (n == 0) return SLA2_OK;
-  const int pairs = (n + 1) / 2;
-  exp2_probe_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return cuda_status(cudaGetLastError());
-}

@@ -303,14 +303,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 #undef SLA2_W8
-// The same 32-bit value into 32 consecutive columns of this thread's lane.
-__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -346,18 +338,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Register reallocation for a warpgroup (all four of its warps execute it):
-// release registers down to N a thread, or wait for the CTA's released
-// registers to raise this warpgroup to N a thread.
-template <int N>
-__device__ __forceinline__ void regs_release() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_claim() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes' worth)
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -382,35 +362,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-// 2^t for two fp32 values at once on the FMA pipe (no MUFU), for t < 128:
-// Cody-Waite style range reduction t = j + f with j = rint(t) and f in
-// [-1/2, 1/2] (the rounding by the 1.5 * 2^23 add), a quartic minimax
-// polynomial for 2^f (coefficients fitted here by the Remez exchange on
-// relative error over [-1/2, 1/2]: max relative error 2.7e-6 with the
-// coefficients rounded to fp32, 2.9e-6 with fp32 Horner steps), and the
-// scaling by 2^j as an integer add to the exponent field. t is clamped below
-// at -125 so that 2^j stays a normal number; the results there (about
-// 2^-125) are below every use of them.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
-  float t0, t1;
-  f2_unpack(t2, t0, t1);
-  t2 = f2_pack(fmaxf(t0, -125.f), fmaxf(t1, -125.f));
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f), neg_magic = f2_pack(-12582912.f, -12582912.f);
-  const uint64_t r = f2_add(t2, magic);                                        // 1.5 * 2^23 + j
-  const uint64_t f = f2_fma(f2_add(r, neg_magic), f2_pack(-1.f, -1.f), t2);    // t - j, exact
-  uint64_t p = f2_fma(f2_pack(0.009570102207362652f, 0.009570102207362652f), f,
-                      f2_pack(0.05591785907745361f, 0.05591785907745361f));
-  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
-  p = f2_fma(p, f, f2_pack(0.6931217908859253f, 0.6931217908859253f));
-  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
-  float r0, r1, p0, p1;
-  f2_unpack(r, r0, r1);
-  f2_unpack(p, p0, p1);
-  // the low bits of r hold j; shifted by 23 they add j to p's exponent
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

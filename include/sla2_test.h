@@ -20,12 +20,6 @@ sla2_status sla2_selftest_timeout(unsigned int* status, unsigned long long budge
  * process; 0 restores the default (2 s). */
 void sla2_set_wait_budget_ns(unsigned long long ns);
 
-/* y[i] = 2^x[i] (i < n) computed the way the sparse branch's softmax computes
- * its share of exponentials on the FMA pipe: range reduction to 2^j * 2^f with
- * f in [-1/2, 1/2] and a cubic polynomial for 2^f (relative error below 1e-4
- * for x in [-125, 128)). x and y are 16-byte aligned device arrays. */
-sla2_status sla2_selftest_exp2(const float* x, float* y, int n, void* stream);
-
 #ifdef __cplusplus
 }
 #endif
