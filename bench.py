@@ -144,9 +144,9 @@ def measured_traffic(name):
 
 def launches_per_forward(w, k):
     """Kernels one forward launches: router 5 (pool, column means, both projections in
-    one launch, logits, top-k), linear state 2, sparse 1, Z_i 1 and epilogue 1 (no Z_i
-    pass when every key block is selected)."""
-    return 5 + 2 + 1 + (2 if k < w.N // 64 else 1)
+    one launch, logits, top-k), linear state 2, sparse 1 and epilogue 1, whatever k."""
+    del w, k
+    return 5 + 2 + 1 + 1
 
 
 class ClockSampler:
@@ -349,6 +349,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--frac", type=float, default=None, help="override k% (sweep)")
+    ap.add_argument("--heads-per-group", type=int, default=2,
+                    help="head group of the end-to-end (host-buffer) leg's copy/compute pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-peaks", action="store_true", help="skip the live 8-bit GEMM peak measurement")
@@ -426,21 +428,22 @@ def main():
     wm = work_model(w, k)
     eff_tops = job_throughput(wm["effective_ops"], ms_step, ws)
 
-    # ---- end to end through the public API: pinned host inputs -> device -> forward -> host output
+    # ---- end to end through the public API: pinned host inputs -> device -> forward -> host
+    # output, one sla2_forward_host call per step (its copies overlap the computation head
+    # group by head group; every step copies all of its inputs in and its output out)
     e2e = None
     if not args.no_e2e:
         host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "proj_q", "proj_k", "alpha")}
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dbuf = {n: torch.empty_like(t[n]) for n in t}
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = hout.numel() * hout.element_size()
+        hpg = max(1, min(args.heads_per_group, w.H))
+        hws = torch.empty(sla2.forward_host_workspace_size(w.B, w.H, w.N, w.d, w.topk_frac, hpg),
+                          dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            for n in host:
-                dbuf[n].copy_(host[n], non_blocking=True)
-            sla2.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["proj_q"], dbuf["proj_k"], dbuf["alpha"],
-                         w.topk_frac, quantize=1, workspace=wsp, out=out, stream=stream)
-            hout.copy_(out, non_blocking=True)
+            sla2.forward_host(host["q"], host["k"], host["v"], host["proj_q"], host["proj_k"], host["alpha"],
+                              w.topk_frac, hout, heads_per_group=hpg, quantize=1, workspace=hws, stream=stream)
 
         for _ in range(2):
             e2e_step()
@@ -459,7 +462,9 @@ def main():
         if ws > 1:
             ms_e2e = max_over_ranks(ms_e2e, dist, dev)
         e2e = {"value": job_throughput(wm["effective_ops"], ms_e2e, ws), "unit": "TOPS",
-               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": f"sla2_forward_host, heads_per_group={hpg}"}
+        del hws
 
     if rank != 0:
         if ws > 1:

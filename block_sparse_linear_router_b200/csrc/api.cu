@@ -55,7 +55,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 // Workspace regions (each 256-byte aligned).
 struct Layout {
   size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
-      htile, hscale, Zi, os, total;
+      htile, hscale, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -93,10 +93,53 @@ Layout make_layout(const Shape& s, int quant) {
   L.Ztot = take(BH * d * 4);
   L.htile = take(BH * d * d * 2);    // fp16 s H_total^T operand tiles
   L.hscale = take(BH * 4);
-  L.Zi = take(BH * nq * d * 4);
-  L.os = take(BH * N * d * 4);
+  L.os = take(BH * N * d * (quant ? 2 : 4));   // fp16 O_s / s_v, or fp32 O_s
   L.total = off;
   return L;
+}
+
+// Workspace of the backward pass: the router's regions, fp32 per-block states,
+// and the gradient accumulators.
+struct BwdLayout {
+  Layout L;          // router and linear-state regions (h: fp32 h_j^T)
+  size_t dos, dHacc, dZacc, dHtot, dZtot, total;
+};
+
+BwdLayout make_bwd_layout(const Shape& s) {
+  BwdLayout B{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t BH = s.BH, d = s.d, nq = s.nq, nk = s.nk, k = s.k, G = s.G;
+  Layout& L = B.L;
+  L.qbar = take(BH * nq * d * 4);
+  L.ksum = take(BH * nk * d * 8);
+  L.c64 = take(BH * d * 8);
+  L.c32 = take(BH * d * 4);
+  L.kbs = take(BH * nk * d * 4);
+  L.A = take(BH * nq * d * 4);
+  L.Bk = take(BH * nk * d * 4);
+  L.scores = take(BH * nq * nk * 4);
+  L.mask = take(BH * nq * nk);
+  L.idx = take(BH * nq * k * 4);
+  L.sq = take(BH * nq * 4);
+  L.vamax = take(BH * d * 4);
+  L.h = take(BH * nk * d * d * 4);
+  L.z = take(BH * nk * d * 4);
+  L.hpart = take(BH * G * d * d * 4);
+  L.zpart = take(BH * G * d * 4);
+  L.Htot = take(BH * d * d * 4);
+  L.Ztot = take(BH * d * 4);
+  B.dos = take(BH * nq * 4);
+  B.dHacc = take(BH * nk * d * d * 4);
+  B.dZacc = take(BH * nk * d * 4);
+  B.dHtot = take(BH * d * d * 4);
+  B.dZtot = take(BH * d * 4);
+  B.total = off;
+  return B;
 }
 
 template <class T>
@@ -214,6 +257,39 @@ cudaError_t aux_stream(AuxStream** out) {
   return cudaSuccess;
 }
 
+// Copy streams and slot events of sla2_forward_host, one set per device,
+// created on the first call there and kept for the life of the process. The
+// slot events are re-recorded for every group; a wait always refers to the
+// latest record, which the enqueue order below makes the right one.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t in_ready[2] = {nullptr, nullptr}, comp_done[2] = {nullptr, nullptr}, out_done[2] = {nullptr, nullptr};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;
+
+cudaError_t host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  HostPipe& p = g_pipe[dev];
+  if (!p.h2d) {
+    cudaStream_t a = nullptr, b = nullptr;
+    if ((e = cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    cudaEvent_t* evs[7] = {&p.start, &p.in_ready[0], &p.in_ready[1], &p.comp_done[0], &p.comp_done[1],
+                           &p.out_done[0], &p.out_done[1]};
+    for (cudaEvent_t* ev : evs)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    p.d2h = b;
+    p.h2d = a;   // set last: a set h2d marks a complete set
+  }
+  *out = &p;
+  return cudaSuccess;
+}
+
 // Clears the caller's status word (if any) on the call's stream, so that a code
 // left there by an earlier call is not read as this call's.
 cudaError_t clear_status(const sla2_desc* d, cudaStream_t st) {
@@ -276,13 +352,6 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   if (r != SLA2_OK) return r;
   SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join
   SLA2_TRY(mark(2));
-  // Z_i (needs the top-k and Z_total) on the auxiliary stream, concurrently with the sparse branch
-  if (s.k < s.nk) {
-    SLA2_TRY(cudaEventRecord(aux->fork, st));
-    SLA2_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
-    SLA2_TRY(launch_zsel(s, at<float>(desc, L.Ztot), at<float>(desc, L.z), idx, at<float>(desc, L.Zi), aux->stream));
-    SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
-  }
 
   // sparse branch: tensor maps over the (quantised) operands
   CUtensorMap tq, tk, tv;
@@ -301,7 +370,9 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
                    CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (!okm) return SLA2_ERR_CUDA;
-  float* os = desc->dbg_os ? desc->dbg_os : at<float>(desc, L.os);
+  // O_s: fp16 O_s / s_v on the quantised path (the epilogue applies s_v and, when asked,
+  // exports fp32 O_s), else fp32 (written straight into the export when there is one)
+  void* os = (!quant && desc->dbg_os) ? static_cast<void*>(desc->dbg_os) : at<void>(desc, L.os);
   SparseArgs sa{idx, at<float>(desc, L.sq), at<float>(desc, L.sk), at<float>(desc, L.sv), os, desc->status, g_budget_ns};
   SLA2_TRY(launch_sparse(s, quant, tq, tk, tv, sa, st));
   SLA2_TRY(mark(3));
@@ -311,9 +382,13 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   ea.htile = at<uint16_t>(desc, L.htile);
   ea.hT = at<uint16_t>(desc, L.h);
   ea.hscale = at<float>(desc, L.hscale);
-  ea.Zi = at<float>(desc, L.Zi);
+  ea.Ztot = at<float>(desc, L.Ztot);
+  ea.z = at<float>(desc, L.z);
   ea.idx = idx;
   ea.os = os;
+  ea.os_half = quant;
+  ea.sv = at<float>(desc, L.sv);
+  ea.os_dbg = quant ? desc->dbg_os : nullptr;
   ea.alpha = alpha;
   ea.H = H;
   ea.out = out;
@@ -321,7 +396,6 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  if (s.k < s.nk) SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join (Z_i)
   SLA2_TRY(launch_epilogue(s, ea, st));
   SLA2_TRY(mark(4));
 
@@ -467,6 +541,76 @@ sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, co
   return forward_body(desc, s, desc->H, L, q, k, v, proj_q, proj_k, alpha, out, st);
 }
 
+size_t sla2_backward_workspace_size(const sla2_desc* desc, float topk_frac) {
+  Shape s;
+  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
+  return make_bwd_layout(s).total;
+}
+
+sla2_status sla2_backward(const sla2_desc* desc, const void* q, const void* k, const void* v, const float* proj_q,
+                          const float* proj_k, const float* alpha, float topk_frac, const float* dout, float* dq,
+                          float* dk, float* dv, float* dalpha, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !dout || !dq || !dk || !dv || !dalpha)
+    return SLA2_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj_q) || !aligned16(proj_k) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SLA2_ERR_INVALID_ARG;
+  const BwdLayout B = make_bwd_layout(s);
+  const Layout& L = B.L;
+  if (!desc->workspace || desc->workspace_bytes < B.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA2_TRY(clear_status(desc, st));
+  // the forward's mask (router) and the per-key-block states (fp32 h_j^T)
+  r = run_router(desc, s, L, q, k, nullptr, proj_q, proj_k, at<uint8_t>(desc, L.mask), at<int32_t>(desc, L.idx), 0,
+                 st);
+  if (r != SLA2_OK) return r;
+  LinearOut o{};
+  o.h = at<void>(desc, L.h);
+  o.h_mode = 0;
+  o.z = at<float>(desc, L.z);
+  o.hpart = at<float>(desc, L.hpart);
+  o.zpart = at<float>(desc, L.zpart);
+  o.quant = 0;
+  o.status = desc->status;
+  o.budget_ns = g_budget_ns;
+  SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, st));
+  SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, nullptr, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
+                                nullptr, nullptr, st));
+  const size_t E = (size_t)s.BH * s.N * s.d;
+  SLA2_TRY(cudaMemsetAsync(dk, 0, E * 4, st));
+  SLA2_TRY(cudaMemsetAsync(dv, 0, E * 4, st));
+  SLA2_TRY(cudaMemsetAsync(dalpha, 0, (size_t)desc->H * s.nq * 4, st));
+  SLA2_TRY(cudaMemsetAsync(at<uint8_t>(desc, B.dHacc), 0, B.total - B.dHacc, st));   // dHacc .. dZtot
+  BackwardArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.c32 = at<float>(desc, L.c32);
+  a.alpha = alpha;
+  a.dout = dout;
+  a.idx = at<int32_t>(desc, L.idx);
+  a.hT = at<float>(desc, L.h);
+  a.z = at<float>(desc, L.z);
+  a.HtotT = at<float>(desc, L.Htot);
+  a.Ztot = at<float>(desc, L.Ztot);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dalpha = dalpha;
+  a.dos_sum = at<float>(desc, B.dos);
+  a.dHacc = at<float>(desc, B.dHacc);
+  a.dZacc = at<float>(desc, B.dZacc);
+  a.dHtot = at<float>(desc, B.dHtot);
+  a.dZtot = at<float>(desc, B.dZtot);
+  SLA2_TRY(launch_backward(s, desc->H, a, st));
+  return SLA2_OK;
+}
+
 size_t sla2_workspace_size_heads(const sla2_desc* desc, int h_count, float topk_frac) {
   Shape s;
   if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
@@ -510,6 +654,124 @@ sla2_status sla2_forward_heads(const sla2_desc* desc, int h_begin, int h_count, 
                      static_cast<const uint16_t*>(v) + e0, pq, pk, al, static_cast<uint8_t*>(out) + e0 * osz, st);
     if (r != SLA2_OK) return r;
   }
+  return SLA2_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of sla2_forward_host: the forward workspace of one group of heads,
+// the projections and alpha of all heads, then two slots of group inputs
+// (Q, K, V) and outputs.
+struct HostLayout {
+  size_t fwd, proj_q, proj_k, alpha, slot[2], in_bytes, out_bytes, total;
+};
+
+HostLayout make_host_layout(const Shape& s, const sla2_desc* d, int hpg) {
+  HostLayout HL{};
+  Shape sh = s;
+  sh.BH = hpg;
+  size_t off = align256(make_layout(sh, d->quantize).total);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t nd = (size_t)s.N * s.d;
+  HL.fwd = 0;
+  HL.proj_q = take((size_t)d->H * s.d * s.d * 4);
+  HL.proj_k = take((size_t)d->H * s.d * s.d * 4);
+  HL.alpha = take((size_t)d->H * s.nq * 4);
+  HL.in_bytes = align256((size_t)hpg * nd * 2);
+  HL.out_bytes = align256((size_t)hpg * nd * (d->out_dtype ? 4 : 2));
+  for (int b = 0; b < 2; ++b) HL.slot[b] = take(3 * HL.in_bytes + HL.out_bytes);
+  HL.total = off;
+  return HL;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sla2_forward_host_workspace_size(const sla2_desc* desc, int heads_per_group, float topk_frac) {
+  Shape s;
+  if (check_desc(desc, topk_frac, &s) != SLA2_OK) return 0;
+  if (heads_per_group < 1 || heads_per_group > desc->H) return 0;
+  return make_host_layout(s, desc, heads_per_group).total;
+}
+
+sla2_status sla2_forward_host(const sla2_desc* desc, int heads_per_group, const void* q, const void* k,
+                              const void* v, const float* proj_q, const float* proj_k, const float* alpha,
+                              float topk_frac, void* out, void* stream) {
+  Shape s;
+  sla2_status r = check_desc(desc, topk_frac, &s);
+  if (r != SLA2_OK) return r;
+  if (heads_per_group < 1 || heads_per_group > desc->H) return SLA2_ERR_INVALID_ARG;
+  if (!q || !k || !v || !proj_q || !proj_k || !alpha || !out) return SLA2_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return SLA2_ERR_INVALID_ARG;
+  if (desc->dbg_scores || desc->dbg_os || desc->dbg_ol || desc->dbg_qhat || desc->dbg_khat || desc->dbg_vhat ||
+      desc->dbg_qscale || desc->dbg_kscale || desc->dbg_vscale || desc->dbg_mask || desc->dbg_idx ||
+      desc->stage_events)
+    return SLA2_ERR_INVALID_ARG;
+  const HostLayout HL = make_host_layout(s, desc, heads_per_group);
+  if (!desc->workspace || desc->workspace_bytes < HL.total ||
+      (reinterpret_cast<uintptr_t>(desc->workspace) & 255u))
+    return SLA2_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> pipe_lock(g_pipe_mu);
+  HostPipe* p = nullptr;
+  SLA2_TRY(host_pipe(&p));
+  SLA2_TRY(clear_status(desc, st));
+  // the copy streams start after everything already enqueued on `stream`
+  // (an earlier call may still be reading the same workspace)
+  SLA2_TRY(cudaEventRecord(p->start, st));
+  SLA2_TRY(cudaStreamWaitEvent(p->h2d, p->start, 0));
+  SLA2_TRY(cudaStreamWaitEvent(p->d2h, p->start, 0));
+  const int H = desc->H;
+  const size_t dd = (size_t)s.d * s.d, nd = (size_t)s.N * s.d, osz = desc->out_dtype ? 4 : 2;
+  float* pq = at<float>(desc, HL.proj_q);
+  float* pk = at<float>(desc, HL.proj_k);
+  float* al = at<float>(desc, HL.alpha);
+  SLA2_TRY(cudaMemcpyAsync(pq, proj_q, (size_t)H * dd * 4, cudaMemcpyHostToDevice, p->h2d));
+  SLA2_TRY(cudaMemcpyAsync(pk, proj_k, (size_t)H * dd * 4, cudaMemcpyHostToDevice, p->h2d));
+  SLA2_TRY(cudaMemcpyAsync(al, alpha, (size_t)H * s.nq * 4, cudaMemcpyHostToDevice, p->h2d));
+  int g = 0;
+  for (int b = 0; b < desc->B; ++b) {
+    for (int h0 = 0; h0 < H; h0 += heads_per_group, ++g) {
+      const int hc = H - h0 < heads_per_group ? H - h0 : heads_per_group;
+      const int sl = g & 1;
+      uint8_t* slot = at<uint8_t>(desc, HL.slot[sl]);
+      uint8_t* dq = slot;
+      uint8_t* dk = slot + HL.in_bytes;
+      uint8_t* dv = slot + 2 * HL.in_bytes;
+      uint8_t* dout = slot + 3 * HL.in_bytes;
+      const size_t e0 = ((size_t)b * H + h0) * nd;   // first element of the group in [B][H][N][d]
+      const size_t in_b = (size_t)hc * nd * 2, out_b = (size_t)hc * nd * osz;
+      // inputs: the slot was last read by the forward of group g - 2
+      if (g >= 2) SLA2_TRY(cudaStreamWaitEvent(p->h2d, p->comp_done[sl], 0));
+      SLA2_TRY(cudaMemcpyAsync(dq, static_cast<const uint8_t*>(q) + e0 * 2, in_b, cudaMemcpyHostToDevice, p->h2d));
+      SLA2_TRY(cudaMemcpyAsync(dk, static_cast<const uint8_t*>(k) + e0 * 2, in_b, cudaMemcpyHostToDevice, p->h2d));
+      SLA2_TRY(cudaMemcpyAsync(dv, static_cast<const uint8_t*>(v) + e0 * 2, in_b, cudaMemcpyHostToDevice, p->h2d));
+      SLA2_TRY(cudaEventRecord(p->in_ready[sl], p->h2d));
+      // compute: the output slot was last copied out for group g - 2
+      SLA2_TRY(cudaStreamWaitEvent(st, p->in_ready[sl], 0));
+      if (g >= 2) SLA2_TRY(cudaStreamWaitEvent(st, p->out_done[sl], 0));
+      Shape sh = s;
+      sh.BH = hc;   // s.G (from all B x H heads) fixes the linear state's summation order
+      const Layout L = make_layout(sh, desc->quantize);
+      r = forward_body(desc, sh, hc, L, dq, dk, dv, pq + (size_t)h0 * dd, pk + (size_t)h0 * dd,
+                       al + (size_t)h0 * s.nq, dout, st);
+      if (r != SLA2_OK) return r;
+      SLA2_TRY(cudaEventRecord(p->comp_done[sl], st));
+      // output
+      SLA2_TRY(cudaStreamWaitEvent(p->d2h, p->comp_done[sl], 0));
+      SLA2_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(out) + e0 * osz, dout, out_b, cudaMemcpyDeviceToHost, p->d2h));
+      SLA2_TRY(cudaEventRecord(p->out_done[sl], p->d2h));
+    }
+  }
+  // `stream` reaches this point once the last output copy (and so every one) is done
+  SLA2_TRY(cudaStreamWaitEvent(st, p->out_done[(g - 1) & 1], 0));
   return SLA2_OK;
 }
 

@@ -5,41 +5,32 @@
 //   O   = alpha_i O_s + (1 - alpha_i) O_l
 // When every key block is selected there is no unselected block and O_l := 0.
 //
-// The numerator never forms H_i: by linearity it is one tensor-core
-// accumulation over k + 1 operand tiles,
-//   D = phi(Q_i) (s H_total) + sum_{j selected} phi(Q_i) (-s h_j)
-// where the linear-state pass stored each -s h_j^T, and the reduce pass
-// s H_total^T, as fp16 d x d tiles already in the 128-byte-swizzled K-major
-// operand layout; s is a per-head power of two that keeps s H_total inside
-// the fp16 range. The denominator phi(Q_i) Z_i is a d-term fp32 dot product
-// per query row, taken while phi is computed; s cancels in O_l = D / (s den).
+// H_i is formed per query block on the CUDA cores: the linear-state pass
+// stored each -s h_j^T, and the reduce pass s H_total^T, as fp16 d x d images
+// already in the 128-byte-swizzled K-major operand layout, so eight "sum"
+// warps add the k + 1 images element by element in fp32 (each thread owns the
+// same 16-byte chunks of every image: coalesced L2 reads, no shared-memory
+// traffic for the gather) and write s H_i^T, rounded once to fp16, as the B
+// operand of ONE tensor-core product D = phi(Q_i) (s H_i) per query block. s is
+// a per-head power of two that keeps s H_total inside the fp16 range. The
+// sum warps also form Z_i = Z_total - sum_sel z_j. The denominator
+// phi(Q_i) Z_i is a d-term fp32 dot product per query row, taken while phi is
+// computed; s cancels in O_l = D / (s den), and so does phi's normalisation
+// (the operand is exp(q - rowmax) without the row sum).
 //
-// The tiles go to the tensor core in groups of G = 256 / d, stacked along N,
-// so that every MMA is 128 x 256 x 16: at that size the tensor pipe hides the
-// per-group barrier wait and commit, which cost a large share of the time of
-// 128 x 128 MMAs. The accumulator then holds G column blocks, one per tile
-// slot, which the readout adds up.
-//
-// Persistent CTAs (one per SM) walk the (head, query block) items in
+// Persistent CTAs (one per SM, 16 warps) walk the (head, query block) items in
 // head-major order, so the SMs work on neighbouring query blocks of the same
-// head and the head's tiles stay in L2. Per CTA:
-//   warps 8,10 producers: each group's tiles, one 1-D bulk copy per tile,
-//              into a ring of shared-memory stages (a single issuing thread
-//              serialises its bulk copies, so two warps share the issue);
-//   warp 9     MMA issuer: per group, d/16 tcgen05 kind::f16 MMAs with
-//              A = phi(Q_i) in tensor memory and B = the stacked tiles, into
-//              the TMEM accumulator, then a commit that frees the stage;
-//   warps 0-7  per item: phi(Q_i), one query row
-//              per thread and half of the features per warp (the two halves
-//              exchange their row max and sum), stored as fp16 into one of two
-//              TMEM A buffers; the denominators phi(Q_i) . Z_i (Z_i precomputed
-//              per query block, copied in by producer 0); then, while the MMAs of this
-//              item run, the readout of the previous item: the accumulator is
-//              read into registers and released at once, then O_l = D / (s den),
-//              the alpha mix with O_s and the store.
-// A lives in tensor memory and Q / O_s go through registers, so shared memory
-// holds only the tile ring and its bandwidth goes to the tiles, each written
-// once by its copy and read once by the MMAs.
+// head and the head's h_j images stay in L2. Per CTA:
+//   warps 8-15 sum: per item, Z_i and s H_i^T (fp16 image) into one of two
+//              shared buffers (the one the MMA of the item before last read);
+//   warps 0-7  per item: exp(Q_i - rowmax), one query row per thread and half
+//              of the features per warp (the two halves exchange their row
+//              max), stored as fp16 into one of two TMEM A buffers, and the
+//              denominators; then thread 0 issues the item's d / 16 tcgen05
+//              kind::f16 MMAs (A from TMEM, B = the s H_i^T image) into one of
+//              two TMEM accumulators and commits; while they run, the warps
+//              read out the previous item: 16 accumulator columns at a time,
+//              O_l = D / (s den), the alpha mix with O_s and the store.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -51,31 +42,30 @@ namespace sla2 {
 namespace {
 
 constexpr int EPI_COMPUTE = 256;          // warps 0-7
-constexpr int EPI_PRODUCER_WARP0 = 8;
-constexpr int EPI_MMA_WARP = 9;
-constexpr int EPI_PRODUCER_WARP1 = 10;
-constexpr int EPI_NPROD = 2;
-constexpr int EPI_THREADS = EPI_COMPUTE + 96;
+constexpr int EPI_SUM_WARP0 = 8;          // warps 8-15
+constexpr int EPI_SUM = 256;
+constexpr int EPI_THREADS = EPI_COMPUTE + EPI_SUM;   // 16 warps: 128 registers a thread
 
 template <int D>
 struct EpiCfg {
-  static constexpr int G = 256 / D;                  // tiles per group (MMA N = 256)
   static constexpr int SLABS = D / 64;               // K slabs of 64 fp16 (128 bytes)
-  static constexpr int TILE = D * D * 2;             // one fp16 operand tile (atom_off layout)
-  static constexpr int SBO = SLABS * 1024;           // bytes between 8-row groups of a tile / group
-  static constexpr int STAGE = G * TILE;             // one ring stage (a group: tiles back to back)
-  static constexpr int NS = (192 * 1024) / STAGE;    // ring stages: 3 (d = 128), 6 (d = 64)
-  static constexpr int HC = D / 2;                   // features (and output columns) per thread
-  static constexpr int OFF_Z = NS * STAGE;                    // Z_i of two items [2][D]
-  static constexpr int OFF_XCH = OFF_Z + 2 * D * 4;           // (max, sum) per row and half [2][BQ]
-  static constexpr int OFF_DEN = OFF_XCH + 2 * BQ * 8;        // denominator halves [2 buffers][2][BQ]
+  static constexpr int TILE = D * D * 2;             // one fp16 operand image (atom_off layout)
+  static constexpr int SBO = SLABS * 1024;           // bytes between 8-row groups of an image
+  static constexpr int CHUNKS = TILE / 16;           // 16-byte chunks of an image
+  static constexpr int CPT = CHUNKS / EPI_SUM;       // chunks per sum thread (8 at d = 128, 2 at d = 64)
+  static constexpr int CPASS = CPT < 4 ? CPT : 4;    // chunks summed per pass (register budget)
+  static constexpr int HC = D / 2;                   // features (and output columns) per compute thread
+  static constexpr int OFF_Z = 2 * TILE;                      // Z_i of two items [2][D]
+  static constexpr int OFF_XCH = OFF_Z + 2 * D * 4;           // row max per half [2][BQ]
+  static constexpr int OFF_DEN = OFF_XCH + 2 * BQ * 4;        // denominator halves [2 buffers][2][BQ]
   static constexpr int OFF_BAR = OFF_DEN + 4 * BQ * 4;
-  static constexpr int NBAR = 2 * NS + 9;
+  static constexpr int NBAR = 11;
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
   static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
-  static_assert(STAGE % 1024 == 0 && OFF_Z % 16 == 0, "bulk-copy and swizzle-atom alignment of the ring");
+  static_assert(TILE % 1024 == 0 && CHUNKS % EPI_SUM == 0 && CPT % CPASS == 0, "image buffers and chunk split");
   static constexpr int KSTEPS = D / 16;              // 16 fp16 (8 TMEM columns of A) per MMA
-  static constexpr uint32_t ACOL = 256;              // A buffers: columns ACOL + b * D / 2
+  static constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, N = D
+  static constexpr uint32_t ACOL = 2 * D;            // accumulators: columns b * D; A buffers: ACOL + b * D / 2
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -89,6 +79,17 @@ __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
 __device__ __forceinline__ uint32_t h2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// acc[0..7] += the eight fp16 values of a 16-byte chunk
+__device__ __forceinline__ void add_h8(float* acc, const uint4& w) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
 }
 
 // Read-only 16-byte load kept where it is written (its latency overlaps the
@@ -106,8 +107,19 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
-// Barrier over the 256 compute threads.
+// Barriers over the 256 compute threads (id 1) and the 256 sum threads (id 2).
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void sum_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
+__device__ __forceinline__ bool sum_sync_any(bool failed) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)failed)
+      : "memory");
+  return r != 0;
+}
 
 // Barrier over the 256 compute threads that also returns, to every one of
 // them, whether any of them passed `failed` (so all take the same exit).
@@ -122,27 +134,76 @@ __device__ __forceinline__ bool compute_sync_any(bool failed) {
   return r != 0;
 }
 
-// O = alpha O_s + (1 - alpha) O_l for 32 consecutive columns of one row
-// (stored with the streaming L2 policy `pol`).
-__device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, float alpha, const float4* osv,
-                                          const float* ol, uint64_t pol) {
-  float o[32];
+// 16 consecutive columns of one row of O_s, at element offset `off` of
+// [BH][N][d], as loaded: four 16-byte words of fp32, or two of fp16 O_s / s_v.
+// The loads are issued here and consumed later by os_convert.
+struct OsChunk {
+  uint4 w[4];
+};
+
+__device__ __forceinline__ void os_issue(const EpilogueArgs& a, size_t off, uint64_t pol, OsChunk& c) {
+  if (a.os_half) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(a.os) + off);
+    c.w[0] = ldg_v4_early(src, pol);
+    c.w[1] = ldg_v4_early(src + 1, pol);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(a.os) + off);
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
-    const float4 v = osv[c / 4];
-    o[c] = alpha * v.x + (1.f - alpha) * ol[c];
-    o[c + 1] = alpha * v.y + (1.f - alpha) * ol[c + 1];
-    o[c + 2] = alpha * v.z + (1.f - alpha) * ol[c + 2];
-    o[c + 3] = alpha * v.w + (1.f - alpha) * ol[c + 3];
+    for (int i = 0; i < 4; ++i) c.w[i] = ldg_v4_early(src + i, pol);
   }
+}
+
+// The chunk as fp32 O_s (fp16 O_s / s_v times s_v of columns col .. col + 15 of
+// head bh), also written to the fp32 export when there is one.
+template <int D>
+__device__ __forceinline__ void os_convert(const EpilogueArgs& a, int bh, size_t off, int col, const OsChunk& c,
+                                           float (&o)[16]) {
+  if (a.os_half) {
+    const float4* sv4 = reinterpret_cast<const float4*>(a.sv + (size_t)bh * D + col);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t u[4] = {c.w[i].x, c.w[i].y, c.w[i].z, c.w[i].w};
+      const float4 s0 = __ldg(sv4 + 2 * i), s1 = __ldg(sv4 + 2 * i + 1);
+      const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[j]));
+        o[i * 8 + 2 * j] = f.x * sv[2 * j];
+        o[i * 8 + 2 * j + 1] = f.y * sv[2 * j + 1];
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[4 * i] = __uint_as_float(c.w[i].x);
+      o[4 * i + 1] = __uint_as_float(c.w[i].y);
+      o[4 * i + 2] = __uint_as_float(c.w[i].z);
+      o[4 * i + 3] = __uint_as_float(c.w[i].w);
+    }
+  }
+  if (a.os_dbg) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 4)
+      *reinterpret_cast<float4*>(a.os_dbg + off + k) = make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+  }
+}
+
+// O = alpha O_s + (1 - alpha) O_l for NC consecutive columns of one row
+// (stored with the streaming L2 policy `pol`).
+template <int NC>
+__device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, float alpha, const float* osv,
+                                          const float* ol, uint64_t pol) {
+  float o[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) o[c] = alpha * osv[c] + (1.f - alpha) * ol[c];
   if (a.ol_dbg) {
 #pragma unroll
-    for (int c = 0; c < 32; c += 4)
+    for (int c = 0; c < NC; c += 4)
       *reinterpret_cast<float4*>(a.ol_dbg + off + c) = make_float4(ol[c], ol[c + 1], ol[c + 2], ol[c + 3]);
   }
   if (a.out_f32) {
 #pragma unroll
-    for (int c = 0; c < 32; c += 4)
+    for (int c = 0; c < NC; c += 4)
       stg_u4_policy(static_cast<float*>(a.out) + off + c,
                     make_uint4(__float_as_uint(o[c]), __float_as_uint(o[c + 1]), __float_as_uint(o[c + 2]),
                                __float_as_uint(o[c + 3])),
@@ -150,7 +211,7 @@ __device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, flo
   } else {
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + off;
 #pragma unroll
-    for (int c = 0; c < 32; c += 8)
+    for (int c = 0; c < NC; c += 8)
       stg_u4_policy(dst + c,
                     make_uint4(cvt_bf16x2(o[c], o[c + 1]), cvt_bf16x2(o[c + 2], o[c + 3]), cvt_bf16x2(o[c + 4], o[c + 5]),
                                cvt_bf16x2(o[c + 6], o[c + 7])),
@@ -163,39 +224,30 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
   using C = EpiCfg<D>;
   extern __shared__ uint8_t esm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = base;
+  uint8_t* hbuf = base;                   // [2] s H_i^T fp16 images
   float* zbuf = reinterpret_cast<float*>(base + C::OFF_Z);
-  float2* xch = reinterpret_cast<float2*>(base + C::OFF_XCH);
+  float* xch = reinterpret_cast<float*>(base + C::OFF_XCH);
   float* den_s = reinterpret_cast<float*>(base + C::OFF_DEN);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
-  uint64_t* empty = full + C::NS;
-  uint64_t* aready = empty + C::NS;       // [2] phi(Q) operand written to TMEM
-  uint64_t* dfull = aready + 2;           // accumulator complete
-  uint64_t* dfree = dfull + 1;            // accumulator read into registers
-  uint64_t* zfull = dfree + 1;            // [2] Z_i of an item landed
-  uint64_t* zfree = zfull + 2;            // [2] Z_i of an item used
-  uint64_t* drain = zfree + 2;
+  uint64_t* hfull = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [2] H_i image and Z_i of an item written
+  uint64_t* hfree = hfull + 2;            // [2] the MMA reading image b has finished
+  uint64_t* dfull = hfull + 4;            // [2] accumulator complete
+  uint64_t* zfree = hfull + 6;            // [2] Z_i of an item used
+  uint64_t* zfull = hfull + 8;            // [2] Z_i of an item written
+  uint64_t* drain = hfull + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(drain + 1) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = s.BH * s.nq;
   const bool has_linear = s.k < s.nk;
-  const int ntile = s.k + 1;
-  const int nblk = ntile < C::G ? ntile : C::G;   // accumulator column blocks in use
 
   if (tid == 0) {
-    for (int i = 0; i < C::NS; ++i) {
-      mbar_init(full + i, EPI_NPROD);
-      mbar_init(empty + i, 1);
-    }
-    mbar_init(aready, EPI_COMPUTE);
-    mbar_init(aready + 1, EPI_COMPUTE);
-    mbar_init(dfull, 1);
-    mbar_init(dfree, EPI_COMPUTE);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(zfull + b, 1);
+      mbar_init(hfull + b, 1);
+      mbar_init(hfree + b, 1);
       mbar_init(zfree + b, EPI_COMPUTE);
+      mbar_init(zfull + b, 1);
+      mbar_init(dfull + b, 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -210,97 +262,67 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == EPI_PRODUCER_WARP0 || warp == EPI_PRODUCER_WARP1) {
-    // ---------------------------------------------------------------- producers
-    const int pr = warp == EPI_PRODUCER_WARP0 ? 0 : 1;   // this producer's tiles: t = pr, pr + 2, ...
-    if (lane == 0 && has_linear) {
-      const size_t tile_elems = (size_t)D * D;
-      const uint64_t keep = l2_policy_evict_last();   // a tile is re-read by ~k query blocks of the head
-      int st = 0, ng = 0, it = 0, nz = 0;
-      uint32_t ph = 0;
+  if (warp >= EPI_SUM_WARP0) {
+    // ---------------------------------------------------------------- sum warps
+    const int st = tid - EPI_SUM_WARP0 * 32;     // 0 .. 255
+    if (has_linear) {
+      const size_t tile_chunks = (size_t)C::CHUNKS;
+      const uint64_t keep = l2_policy_evict_last();   // an image is re-read by ~k query blocks of the head
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
+      int it = 0;
+      for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
         const int bh = w / s.nq, qi = w % s.nq;
-        const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * s.k;
-        if (pr == 0) {   // Z_i of this item (its buffer was last read for item it - 2)
-          const int b = it & 1;
-          if (it >= 2 && !mbar_wait(zfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(zfull + b, D * 4);
-          bulk_load(zbuf + b * D, a.Zi + ((size_t)bh * s.nq + qi) * D, D * 4, zfull + b);
-          ++nz;
-        }
-        for (int n0 = 0; n0 < ntile; n0 += C::G) {
-          const int cnt = ntile - n0 < C::G ? ntile - n0 : C::G;
-          if (ng >= C::NS && !mbar_wait(empty + st, ph ^ 1u, abort_flag, a.status, a.budget_ns)) {
-            ok = false;
-            break;
-          }
-          const int mine = cnt > pr ? (cnt - pr + EPI_NPROD - 1) / EPI_NPROD : 0;
-          mbar_arrive_expect_tx(full + st, (uint32_t)(mine * C::TILE));
-          uint8_t* dst = ring + st * C::STAGE;
-          for (int t = pr; t < cnt; t += EPI_NPROD) {
-            const int n = n0 + t;
-            const uint16_t* src = n == 0 ? a.htile + (size_t)bh * tile_elems
-                                         : a.hT + ((size_t)bh * s.nk + __ldg(sel + n - 1)) * tile_elems;
-            bulk_load_hint(dst + t * C::TILE, src, C::TILE, full + st, keep);
-          }
-          ++ng;
-          if (++st == C::NS) {
-            st = 0;
-            ph ^= 1u;
-          }
-        }
-      }
-      if (!ok) {   // let the copies in flight land before the CTA's shared memory is released
-        for (int q = (ng > C::NS ? ng - C::NS : 0); q < ng; ++q)
-          mbar_wait_drain(full + q % C::NS, (q / C::NS) & 1, 20000000ull);
-        for (int q = (nz > 2 ? nz - 2 : 0); q < nz; ++q) mbar_wait_drain(zfull + (q & 1), (q >> 1) & 1, 20000000ull);
-      }
-    }
-    __syncwarp();
-  } else if (warp == EPI_MMA_WARP) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && has_linear) {
-      const uint64_t bdesc0 = make_sdesc(smem_u32(ring), C::SBO, LAYOUT_SW128);
-      int st = 0, it = 0;
-      uint32_t ph = 0;
-      bool ok = true, issued = false;
-      for (int w = blockIdx.x; ok && w < total; w += gridDim.x, ++it) {
         const int b = it & 1;
-        if (!mbar_wait(aready + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
-        if (it >= 1 && !mbar_wait(dfree, (it - 1) & 1, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t acol = tmem + C::ACOL + (uint32_t)(b * (D / 2));
-        for (int n0 = 0; n0 < ntile; n0 += C::G) {
-          const int cnt = ntile - n0 < C::G ? ntile - n0 : C::G;
-          const uint32_t idesc = make_idesc(1, 0, 0, 128, (uint32_t)(cnt * D));   // fp16 x fp16 -> fp32
-          if (!mbar_wait(full + st, ph, abort_flag, a.status, a.budget_ns)) { ok = false; break; }
-          tc_fence_after();
-          // descriptor start addresses advance in 16-byte units
-          const uint64_t bd = bdesc0 + (uint64_t)((st * C::STAGE) >> 4);
-#pragma unroll
-          for (int ks = 0; ks < C::KSTEPS; ++ks)
-            mma_f16_ts(tmem, acol + ks * 8, bd + (uint64_t)(((ks >> 2) * 1024 + (ks & 3) * 32) >> 4), idesc,
-                       (n0 | ks) != 0);
-          issued = true;
-          tc_commit(empty + st);
-          if (++st == C::NS) {
-            st = 0;
-            ph ^= 1u;
-          }
+        const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * s.k;
+        // the image and Z_i buffers b were last read for item it - 2
+        bool okw = true;
+        if (it >= 2) {
+          okw = mbar_wait(hfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns) &&
+                mbar_wait(zfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns);
         }
-        if (!ok) break;
-        tc_commit(dfull);
+        if (sum_sync_any(!okw)) { ok = false; break; }
+        // Z_i = Z_total - the selected z_j, in ascending block order
+        if (st < D) {
+          float acc = a.Ztot[(size_t)bh * D + st];
+          for (int n = 0; n < s.k; ++n) acc -= a.z[((size_t)bh * s.nk + __ldg(sel + n)) * D + st];
+          zbuf[b * D + st] = acc;
+        }
+        sum_sync();
+        if (st == 0) mbar_arrive(zfull + b);
+        // s H_i^T = s H_total^T + sum of the selected -s h_j^T, chunk by chunk
+        const uint4* img0 = reinterpret_cast<const uint4*>(a.htile + (size_t)bh * D * D);
+        const uint4* imgs = reinterpret_cast<const uint4*>(a.hT);
+        uint4* dst = reinterpret_cast<uint4*>(hbuf + b * C::TILE);
+#pragma unroll 1
+        for (int pass = 0; pass < C::CPT / C::CPASS; ++pass) {
+          float acc[C::CPASS * 8];
+#pragma unroll
+          for (int c = 0; c < C::CPASS * 8; ++c) acc[c] = 0.f;
+          const int c0 = st + pass * C::CPASS * EPI_SUM;
+#pragma unroll
+          for (int c = 0; c < C::CPASS; ++c) add_h8(acc + c * 8, ldg_v4_early(img0 + c0 + c * EPI_SUM, keep));
+          int j_next = __ldg(sel);
+          for (int n = 0; n < s.k; ++n) {
+            const int j = j_next;
+            if (n + 1 < s.k) j_next = __ldg(sel + n + 1);
+            const uint4* img = imgs + ((size_t)bh * s.nk + j) * tile_chunks;
+            uint4 w4[C::CPASS];
+#pragma unroll
+            for (int c = 0; c < C::CPASS; ++c) w4[c] = ldg_v4_early(img + c0 + c * EPI_SUM, keep);
+#pragma unroll
+            for (int c = 0; c < C::CPASS; ++c) add_h8(acc + c * 8, w4[c]);
+          }
+#pragma unroll
+          for (int c = 0; c < C::CPASS; ++c)
+            dst[c0 + c * EPI_SUM] = make_uint4(h2(acc[c * 8], acc[c * 8 + 1]), h2(acc[c * 8 + 2], acc[c * 8 + 3]),
+                                               h2(acc[c * 8 + 4], acc[c * 8 + 5]), h2(acc[c * 8 + 6], acc[c * 8 + 7]));
+        }
+        fence_proxy_async_smem();
+        sum_sync();
+        if (st == 0) mbar_arrive(hfull + b);
       }
-      if (!ok && issued) {   // issued MMAs finish before the CTA releases TMEM and shared memory
-        tc_commit(drain);
-        mbar_wait_drain(drain, 0, 20000000ull);
-      }
+      (void)ok;
     }
-    __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warps
     constexpr int HC = C::HC;
@@ -312,67 +334,55 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
     auto row_of = [&](int w) { return (size_t)(w / s.nq) * s.N + (size_t)(w % s.nq) * BQ + r; };
 
     if (!has_linear) {
-      float zero[32];
+      float zero[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) zero[c] = 0.f;
+      for (int c = 0; c < 16; ++c) zero[c] = 0.f;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         const int bh = w / s.nq, qi = w % s.nq;
         const float alpha = a.alpha[(size_t)(bh % a.H) * s.nq + qi];
         const size_t row = row_of(w);
 #pragma unroll
-        for (int cc = 0; cc < HC / 32; ++cc) {
-          float4 osv[8];
-          const float4* osr = reinterpret_cast<const float4*>(a.os + row * D + fh * HC + cc * 32);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) osv[c] = __ldg(osr + c);
-          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, zero, stream_pol);
+        for (int cc = 0; cc < HC / 16; ++cc) {
+          const size_t off = row * D + fh * HC + cc * 16;
+          OsChunk ch;
+          os_issue(a, off, stream_pol, ch);
+          float osv[16];
+          os_convert<D>(a, bh, off, fh * HC + cc * 16, ch, osv);
+          mix_store<16>(a, off, alpha, osv, zero, stream_pol);
         }
       }
     } else {
-      // readout of item `itp` (work index wp): the accumulator's column blocks
-      // summed into registers, the accumulator released, then O_l, mix, store
+      // readout of item `itp` (work index wp): 16 accumulator columns at a
+      // time scaled to O_l, mixed with O_s and stored; the accumulator is
+      // released after its last columns are read
       auto readout = [&](int itp, int wp) -> bool {
         const int bh = wp / s.nq, qi = wp % s.nq;
         const float alpha = a.alpha[(size_t)(bh % a.H) * s.nq + qi];
         const float hsc = a.hscale[bh];
         const size_t row = row_of(wp);
         const int bp = itp & 1;
-        const float* osr = a.os + row * D + fh * HC;
-        float4 osv[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) osv[c] = ldg_f4_policy(reinterpret_cast<const float4*>(osr) + c, stream_pol);
-        bool ok = mbar_wait(dfull, itp & 1, abort_flag, a.status, a.budget_ns);
+        const size_t off0 = row * D + fh * HC;
+        OsChunk ch[2];
+        os_issue(a, off0, stream_pol, ch[0]);   // in flight during the wait
+        bool ok = mbar_wait(dfull + bp, (itp >> 1) & 1, abort_flag, a.status, a.budget_ns);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (!ok) return false;
-        float ol[HC];
-#pragma unroll
-        for (int cc = 0; cc < HC / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + (uint32_t)(fh * HC + cc * 32), v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) ol[cc * 32 + c] = __uint_as_float(v[c]);
-          for (int blk = 1; blk < nblk; ++blk) {
-            tmem_ld32(tmem + lane_base + (uint32_t)(blk * D + fh * HC + cc * 32), v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) ol[cc * 32 + c] += __uint_as_float(v[c]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(dfree);
         const float inv = 1.f / (hsc * (den_s[(bp * 2) * BQ + r] + den_s[(bp * 2 + 1) * BQ + r]));
 #pragma unroll
-        for (int c = 0; c < HC; ++c) ol[c] *= inv;
+        for (int cc = 0; cc < HC / 16; ++cc) {
+          if (cc + 1 < HC / 16) os_issue(a, off0 + (cc + 1) * 16, stream_pol, ch[(cc + 1) & 1]);
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + (uint32_t)(bp * D + fh * HC + cc * 16), v);
+          tmem_wait_ld();
+          float osv[16];
+          os_convert<D>(a, bh, off0 + cc * 16, fh * HC + cc * 16, ch[cc & 1], osv);
+          float ol[16];
 #pragma unroll
-        for (int cc = 0; cc < HC / 32; ++cc) {
-          if (cc > 0) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) osv[c] = ldg_f4_policy(reinterpret_cast<const float4*>(osr + cc * 32) + c, stream_pol);
-          }
-          mix_store(a, row * D + fh * HC + cc * 32, alpha, osv, ol + cc * 32, stream_pol);
+          for (int c = 0; c < 16; ++c) ol[c] = __uint_as_float(v[c]) * inv;
+          mix_store<16>(a, off0 + cc * 16, alpha, osv, ol, stream_pol);
         }
+        tc_fence_before();   // the reads are ordered before the next compute barrier (the MMA that reuses it)
         return true;
       };
 
@@ -384,50 +394,38 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
       };
       load_q(blockIdx.x);
       int it = 0, wprev = -1;
-      bool ok = true, rd_ok = true;
+      bool ok = true, rd_ok = true, issued = false;
       for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
         const int bh = w / s.nq, qi = w % s.nq;
         const int b = it & 1;
         if (wprev >= 0) {                        // O_s of the previous item, read out below
-          const float* p = a.os + row_of(wprev) * D + fh * HC;
-#pragma unroll
-          for (int c = 0; c < HC; c += 32) prefetch_l2(p + c);
+          const size_t esz = a.os_half ? 2 : 4;
+          const uint8_t* p = static_cast<const uint8_t*>(a.os) + (row_of(wprev) * D + fh * HC) * esz;
+          for (int c = 0; c < (int)(HC * esz); c += 128) prefetch_l2(p + c);
         }
         (void)bh;
         (void)qi;
-        // ---- phi = softmax over the d features: local max / sum, then exchanged between the halves
-        float x[HC];
-#pragma unroll
-        for (int q = 0; q < HC / 8; ++q) {
-          float v8[8];
-          unpack8(qv[q], v8);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) x[q * 8 + c] = v8[c];
-        }
+        // ---- phi = softmax over the d features. Its normalisation cancels in
+        // O_l = phi H_i / (phi Z_i), so the operand is e = exp(q - M) with M
+        // the row max (exchanged between the two halves) and no row sum.
+        float m4[4];
         {
-          const int wn = w + gridDim.x;          // the next item's Q rows, consumed next iteration
-          if (wn < total) load_q(wn);
-        }
-        // four independent partial chains for the max and the sum
-        float m4[4] = {x[0], x[1], x[2], x[3]};
+          float v8[8];
+          unpack8(qv[0], v8);
+          m4[0] = fmaxf(v8[0], v8[4]); m4[1] = fmaxf(v8[1], v8[5]);
+          m4[2] = fmaxf(v8[2], v8[6]); m4[3] = fmaxf(v8[3], v8[7]);
 #pragma unroll
-        for (int c = 4; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
+          for (int q = 1; q < HC / 8; ++q) {
+            unpack8(qv[q], v8);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) m4[c & 3] = fmaxf(m4[c & 3], v8[c]);
+          }
+        }
         const float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        const float mb = m * kLog2e;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          x[c] = ex2_approx(fmaf(x[c], kLog2e, -mb));
-          s4[c & 3] += x[c];
-        }
-        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        xch[fh * BQ + r] = make_float2(m, sum);
+        xch[fh * BQ + r] = m;
         compute_sync();
-        const float2 o = xch[(fh ^ 1) * BQ + r];
-        const float M = fmaxf(m, o.x);
-        const float e_own = ex2_approx((m - M) * kLog2e);
-        const float scale = e_own / (sum * e_own + o.y * ex2_approx((o.x - M) * kLog2e));
-        // den = phi(Q_i) . Z_i over this half of the features
+        const float mb = fmaxf(m, xch[(fh ^ 1) * BQ + r]) * kLog2e;
+        // den = e . Z_i over this half of the features
         bool zok = mbar_wait(zfull + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns);
         zok = __all_sync(0xffffffffu, zok);
         ok = ok && zok;
@@ -435,15 +433,21 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         float d4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[HC / 2];
 #pragma unroll
-        for (int c = 0; c < HC; c += 4) {
-          const float4 zz = zok ? zi4[c / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float p0 = x[c] * scale, p1 = x[c + 1] * scale, p2 = x[c + 2] * scale, p3 = x[c + 3] * scale;
-          d4[0] = fmaf(p0, zz.x, d4[0]);
-          d4[1] = fmaf(p1, zz.y, d4[1]);
-          d4[2] = fmaf(p2, zz.z, d4[2]);
-          d4[3] = fmaf(p3, zz.w, d4[3]);
-          pk[c / 2] = h2(p0, p1);
-          pk[c / 2 + 1] = h2(p2, p3);
+        for (int q = 0; q < HC / 8; ++q) {
+          float v8[8];
+          unpack8(qv[q], v8);
+#pragma unroll
+          for (int c = 0; c < 8; c += 4) {
+            const float4 zz = zok ? zi4[(q * 8 + c) / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float p0 = ex2_approx(fmaf(v8[c], kLog2e, -mb)), p1 = ex2_approx(fmaf(v8[c + 1], kLog2e, -mb));
+            const float p2 = ex2_approx(fmaf(v8[c + 2], kLog2e, -mb)), p3 = ex2_approx(fmaf(v8[c + 3], kLog2e, -mb));
+            d4[0] = fmaf(p0, zz.x, d4[0]);
+            d4[1] = fmaf(p1, zz.y, d4[1]);
+            d4[2] = fmaf(p2, zz.z, d4[2]);
+            d4[3] = fmaf(p3, zz.w, d4[3]);
+            pk[(q * 8 + c) / 2] = h2(p0, p1);
+            pk[(q * 8 + c) / 2 + 1] = h2(p2, p3);
+          }
         }
         mbar_arrive(zfree + b);
         den_s[(b * 2 + fh) * BQ + r] = (d4[0] + d4[1]) + (d4[2] + d4[3]);
@@ -455,14 +459,39 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(aready + b);
-        // every compute thread takes this exit together
+        {
+          const int wn = w + gridDim.x;          // the next item's Q rows, consumed next iteration
+          if (wn < total) load_q(wn);
+        }
+        // every compute thread takes this exit together; past it, the phi operand is in
+        // TMEM and the readout of item it - 2 (same accumulator) is complete
         if (compute_sync_any(!ok || !rd_ok)) { ok = false; break; }
+        if (tid == 0) {   // MMA issue: D_b = phi(Q_i) (s H_i) once the sum warps have written s H_i^T
+          tc_fence_after();
+          if (mbar_wait(hfull + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns)) {
+            tc_fence_after();
+            const uint32_t acol = tmem + C::ACOL + (uint32_t)(b * (D / 2));
+            const uint64_t bd = make_sdesc(smem_u32(hbuf + b * C::TILE), C::SBO, LAYOUT_SW128);
+#pragma unroll
+            for (int ks = 0; ks < C::KSTEPS; ++ks)
+              mma_f16_ts(tmem + (uint32_t)(b * D), acol + ks * 8,
+                         bd + (uint64_t)(((ks >> 2) * 1024 + (ks & 3) * 32) >> 4), C::IDESC, ks != 0);
+            issued = true;
+            tc_commit(hfree + b);
+            tc_commit(dfull + b);
+          } else {
+            ok = false;     // seen by every compute thread at the next barrier; the readout's wait fails first
+          }
+        }
         // ---- the previous item's readout overlaps this item's MMAs
         if (wprev >= 0) rd_ok = readout(it - 1, wprev);
         wprev = w;
       }
-      if (ok && rd_ok && wprev >= 0) readout(it - 1, wprev);
+      if (ok && rd_ok && wprev >= 0) rd_ok = readout(it - 1, wprev);
+      if (tid == 0 && issued && !(ok && rd_ok)) {   // issued MMAs finish before TMEM and shared memory are released
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0, 20000000ull);
+      }
     }
   }
   tc_fence_before();
@@ -473,27 +502,9 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
   }
 }
 
-// Z_i = Z_total - sum of the selected z_j for every (head, query block), one
-// feature per thread, the selected blocks in ascending order.
-__global__ void zsel_kernel(const float* __restrict__ Ztot, const float* __restrict__ z, const int32_t* __restrict__ idx,
-                            int nq, int nk, int k, float* __restrict__ Zi) {
-  const int qi = blockIdx.x, bh = blockIdx.y, c = threadIdx.x, D = blockDim.x;
-  const int32_t* sel = idx + ((size_t)bh * nq + qi) * k;
-  float acc = Ztot[(size_t)bh * D + c];
-#pragma unroll 8
-  for (int n = 0; n < k; ++n) acc -= z[((size_t)bh * nk + __ldg(sel + n)) * D + c];
-  Zi[((size_t)bh * nq + qi) * D + c] = acc;
-}
-
 constexpr int kSMs = 148;   // B200 streaming multiprocessors
 
 }  // namespace
-
-cudaError_t launch_zsel(const Shape& s, const float* Ztot, const float* z, const int32_t* idx, float* Zi,
-                        cudaStream_t st) {
-  zsel_kernel<<<dim3(s.nq, s.BH), s.d, 0, st>>>(Ztot, z, idx, s.nq, s.nk, s.k, Zi);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st) {
   const int total = s.BH * s.nq;

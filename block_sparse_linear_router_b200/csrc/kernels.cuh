@@ -87,7 +87,7 @@ struct SparseArgs {
   const float* sq;      // [BH][nq]   (quant)
   const float* sk;      // [BH][nk]   (quant)
   const float* sv;      // [BH][d]    (quant)
-  float* os;            // [BH][N][d] fp32 out
+  void* os;             // [BH][N][d] out: fp32 O_s, or (quant) fp16 O_s / s_v (magnitudes <= 448)
   unsigned* status;
   unsigned long long budget_ns;
 };
@@ -102,9 +102,13 @@ struct EpilogueArgs {
   const uint16_t* htile;  // fp16 s H_total^T operand images [BH][d*d] (h_mode-2 layout)
   const uint16_t* hT;     // fp16 -s h_j^T operand images [BH][nk][d*d] (h_mode 2)
   const float* hscale;    // [BH] s
-  const float* Zi;        // [BH][nq][d] Z_total - sum of the selected z_j
+  const float* Ztot;      // [BH][d] Z_total
+  const float* z;         // [BH][nk][d] z_j
   const int32_t* idx;     // [BH][nq][k]
-  const float* os;        // [BH][N][d]
+  const void* os;         // [BH][N][d] O_s: fp32, or fp16 O_s / s_v when os_half
+  int os_half;
+  const float* sv;        // [BH][d] s_v (os_half)
+  float* os_dbg;          // optional [BH][N][d] fp32 O_s export
   const float* alpha;     // [H][nq]
   int H;
   void* out;              // [BH][N][d]
@@ -113,9 +117,31 @@ struct EpilogueArgs {
   unsigned* status;
   unsigned long long budget_ns;
 };
-// Z_i per (head, query block), the epilogue's denominators' second factor
-cudaError_t launch_zsel(const Shape& s, const float* Ztot, const float* z, const int32_t* idx, float* Zi,
-                        cudaStream_t st);
 cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st);
+
+// ---- backward pass (backward.cu) ------------------------------------------
+struct BackwardArgs {
+  const void* q;          // bf16 [BH][N][d]
+  const void* k;
+  const void* v;
+  const float* c32;       // colmean of K, [BH][d]
+  const float* alpha;     // [H][nq]
+  const float* dout;      // dL/dO, fp32 [BH][N][d]
+  const int32_t* idx;     // selected key blocks [BH][nq][k]
+  const float* hT;        // h_j^T fp32 [BH][nk][d][d] (channel, feature)
+  const float* z;         // z_j [BH][nk][d]
+  const float* HtotT;     // H_total^T [BH][d][d]
+  const float* Ztot;      // Z_total [BH][d]
+  float* dq;              // outputs, fp32 [BH][N][d]
+  float* dk;              // zeroed by the caller (accumulates dK_s, then dK)
+  float* dv;              // zeroed by the caller
+  float* dalpha;          // [H][nq], zeroed by the caller (summed over the batch)
+  float* dos_sum;         // [BH][nq] scratch
+  float* dHacc;           // [BH][nk][d][d] scratch, zeroed
+  float* dZacc;           // [BH][nk][d] scratch, zeroed
+  float* dHtot;           // [BH][d][d] scratch, zeroed
+  float* dZtot;           // [BH][d] scratch, zeroed
+};
+cudaError_t launch_backward(const Shape& s, int H, const BackwardArgs& a, cudaStream_t st);
 
 }  // namespace sla2

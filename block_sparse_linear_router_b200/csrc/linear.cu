@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
 // H_total^T and Z_total as fixed-order sums of the chunk partials. With vamax
 // given, also the head's fp16 scale s (the same value the linear-state pass
 // used for its h_j tiles) and s H_total^T as an fp16 operand image in the
-// h_mode-2 layout, which the epilogue loads as the first B tile of every item.
+// h_mode-2 layout, to which the epilogue adds the selected blocks' images.
 __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const float* __restrict__ zpart, int G, int D,
                                      int N, const unsigned* __restrict__ vamax, float* __restrict__ Htot,
                                      float* __restrict__ Ztot, uint16_t* __restrict__ htile,

@@ -13,7 +13,10 @@
 //              softmax with one running-max update per key block; P written
 //              to shared memory as e4m3 (x448 fixed scale) or bf16; O rescaled
 //              in TMEM when a row max grows; at the end of an item the row is
-//              normalised and stored while the next item's S is computed.
+//              normalised and stored while the next item's S is computed (fp32
+//              O_s, or on the quantised path the fp16 row O_s / s_v: a
+//              weighted mean of e4m3 V-hat codes, so |.| <= 448 and the
+//              epilogue applies s_v).
 //   warp 4     TMA producer: per item the Q tile (double-buffered, prefetched
 //              one item ahead); K_j and V_j^T of each selected j into separate
 //              rings of NS stages (no multicast): a K stage is released when
@@ -25,6 +28,7 @@
 //              O += P_g V_j (kind::f8f6f4 e4m3 or kind::f16 bf16 -> f32).
 // TMEM columns: [0,64) S buffer 0, [64,128) S buffer 1, [128,128+D) O.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "device.cuh"
 #include "kernels.cuh"
@@ -79,6 +83,11 @@ __device__ __forceinline__ uint32_t kstep_addr(uint32_t tile, int rows, int ks) 
 }
 
 constexpr uint64_t DRAIN_NS = 20000000ull;   // 20 ms for in-flight copies / MMAs after an abort
+
+__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
 template <int D, bool QUANT>
 __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid_constant__ CUtensorMap tq,
@@ -455,22 +464,30 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.f / l;     // quantised path: l holds 448 x the row sum
-      float* orow = a.os + ((size_t)bh * s.N + (size_t)qi * BQ + r) * D;
-      const float* svh = a.sv + (size_t)bh * D;
+      const size_t orow = ((size_t)bh * s.N + (size_t)qi * BQ + r) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32(lane_addr + C::COL_O + cc * 32, o);
         tmem_wait_ld();
-        float v[32];
+        if constexpr (QUANT) {
+          // O_s / s_v = acc / l: a weighted mean of V-hat codes, |.| <= 448, stored as fp16
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(a.os) + orow + cc * 32);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float acc = __uint_as_float(o[c]);
-          v[c] = QUANT ? acc * __ldg(svh + cc * 32 + c) * inv_l : acc * inv_l;
+          for (int c = 0; c < 32; c += 8)
+            dst[c / 8] = make_uint4(
+                h2_bits(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l),
+                h2_bits(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l),
+                h2_bits(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l),
+                h2_bits(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l));
+        } else {
+          float* dst = static_cast<float*>(a.os) + orow + cc * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
+                            __uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
         }
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          *reinterpret_cast<float4*>(orow + cc * 32 + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
       }
       tc_fence_before();
       __syncwarp();

@@ -55,8 +55,14 @@ SIGNATURES = {
     "sla2_forward": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 6 + [ctypes.c_float]
                      + [ctypes.c_void_p] * 2),
     "sla2_workspace_size_heads": (ctypes.c_size_t, [ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_float]),
+    "sla2_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Desc), ctypes.c_float]),
+    "sla2_backward": (ctypes.c_int, [ctypes.POINTER(Desc)] + [ctypes.c_void_p] * 6 + [ctypes.c_float]
+                      + [ctypes.c_void_p] * 6),
     "sla2_forward_heads": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 6
                            + [ctypes.c_float] + [ctypes.c_void_p] * 2),
+    "sla2_forward_host_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Desc), ctypes.c_int, ctypes.c_float]),
+    "sla2_forward_host": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.c_int] + [ctypes.c_void_p] * 6
+                          + [ctypes.c_float] + [ctypes.c_void_p] * 2),
 }
 
 _lib = None
@@ -289,3 +295,68 @@ def forward_heads(q, k, v, proj_q, proj_k, alpha, frac, h_begin, h_count, out, q
     if r != 0:
         raise Sla2Error(r, "sla2_forward_heads")
     return out
+
+
+def forward_host_workspace_size(B, H, N, d, frac, heads_per_group, quantize=1, out_dtype=torch.bfloat16) -> int:
+    desc = make_desc(B, H, N, d, quantize, 1 if out_dtype == torch.float32 else 0)
+    return load_library().sla2_forward_host_workspace_size(ctypes.byref(desc), heads_per_group, frac)
+
+
+def forward_host(q, k, v, proj_q, proj_k, alpha, frac, out, heads_per_group=2, quantize=1,
+                 workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, stream=None):
+    """The forward pass from HOST tensors to the HOST tensor `out` (bf16 or fp32 [B,H,N,d]),
+    with the copies overlapped with the computation head group by head group; the
+    workspace is device memory. Returns once enqueued: `out` is complete when `stream`
+    (default: the current stream) is, and the host tensors must live until then
+    (page-locked tensors let the copies run asynchronously)."""
+    lib = load_library()
+    for t in (q, k, v, proj_q, proj_k, alpha, out):
+        if t.is_cuda:
+            raise ValueError("forward_host takes host tensors")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    B, H, N, d = q.shape
+    if out.dtype not in (torch.bfloat16, torch.float32) or tuple(out.shape) != (B, H, N, d):
+        raise ValueError("out must be a bf16 or fp32 [B,H,N,d] tensor")
+    f32 = 1 if out.dtype == torch.float32 else 0
+    desc = make_desc(B, H, N, d, quantize, f32)
+    n = lib.sla2_forward_host_workspace_size(ctypes.byref(desc), heads_per_group, frac)
+    if n == 0:
+        raise Sla2Error(1, "sla2_forward_host_workspace_size")
+    ws = workspace if workspace is not None else torch.empty(n, dtype=torch.uint8, device="cuda")
+    if not ws.is_cuda:
+        raise ValueError("the workspace is device memory")
+    desc.workspace, desc.workspace_bytes = ws.data_ptr(), ws.numel()
+    if status is not None:
+        desc.status = status.data_ptr()
+    r = lib.sla2_forward_host(ctypes.byref(desc), heads_per_group, _ptr(q), _ptr(k), _ptr(v), _ptr(proj_q),
+                              _ptr(proj_k), _ptr(alpha), frac, _ptr(out), _stream(stream))
+    if r != 0:
+        raise Sla2Error(r, "sla2_forward_host")
+    return out
+
+
+def backward(q, k, v, proj_q, proj_k, alpha, frac, dout, workspace: Optional[torch.Tensor] = None,
+             status: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of the unquantised forward for the router's mask: (dq, dk, dv) fp32
+    [B,H,N,d] and dalpha fp32 [H,nq] (summed over the batch), for dL/dO = dout (fp32)."""
+    lib = load_library()
+    _check_qkv(q, k, v, proj_q, proj_k, alpha, dout)
+    if dout.dtype != torch.float32 or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("dout must be fp32 with the shape of q")
+    B, H, N, d = q.shape
+    desc = make_desc(B, H, N, d, 0)
+    n = lib.sla2_backward_workspace_size(ctypes.byref(desc), frac)
+    if n == 0:
+        raise Sla2Error(1, "sla2_backward_workspace_size")
+    ws = workspace if workspace is not None else torch.empty(n, dtype=torch.uint8, device=q.device)
+    desc.workspace, desc.workspace_bytes = ws.data_ptr(), ws.numel()
+    if status is not None:
+        desc.status = status.data_ptr()
+    dq, dk, dv = (torch.empty(B, H, N, d, dtype=torch.float32, device=q.device) for _ in range(3))
+    dalpha = torch.empty(H, N // 128, dtype=torch.float32, device=q.device)
+    r = lib.sla2_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(proj_q), _ptr(proj_k), _ptr(alpha),
+                          frac, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _stream(stream))
+    if r != 0:
+        raise Sla2Error(r, "sla2_backward")
+    return dq, dk, dv, dalpha

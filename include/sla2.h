@@ -181,8 +181,7 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
  * All intermediates live in desc->workspace; optional debug exports in desc.
  * The linear-state pass runs on a library-owned non-blocking stream, forked
  * from and joined back into `stream` with events, concurrently with the
- * router's projections, logits and top-k on `stream`; the Z_i pass runs on it
- * too, concurrently with the sparse branch. That stream and its two events are
+ * router's projections, logits and top-k on `stream`. That stream and its two events are
  * created by the first call on each device and kept until the process exits;
  * make that first call outside any stream capture. Later calls can be captured
  * (the fork and join become graph edges). Calls from several host threads are
@@ -195,6 +194,57 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
 sla2_status sla2_forward(const sla2_desc* desc, const void* q, const void* k, const void* v,
                          const float* proj_q, const float* proj_k, const float* alpha,
                          float topk_frac, void* out, void* stream);
+
+/* Backward pass (detail page §7 note 3: the hand-derived gradient with the
+ * linear branch's dH_i and dZ_i formed once per query block; §2 table: the
+ * backward runs at higher precision than the INT8/FP8 forward kernels). It is
+ * the gradient of the UNQUANTISED forward O = alpha O_s + (1 - alpha) O_l for
+ * the mask the router selects for these inputs, held fixed (the hard Top-k is
+ * piecewise constant, so proj_q and proj_k receive no gradient on this path),
+ * with K smoothing included.
+ *   q, k, v     : bf16 [B][H][N][d] (the forward's inputs); proj_q/proj_k,
+ *                 alpha, topk_frac as for sla2_forward
+ *   dout        : fp32 [B][H][N][d], dL/dO
+ *   dq, dk, dv  : fp32 [B][H][N][d], written (not accumulated)
+ *   dalpha      : fp32 [H][N/128], dL/dalpha summed over the batch (alpha is
+ *                 shared over the batch), written
+ * Arithmetic: fp32 on the CUDA cores; the per-key-block states h_j come from
+ * the linear-state pass (fp16 tensor-core operands, fp32 accumulation).
+ * Workspace: sla2_backward_workspace_size bytes; desc->quantize, out_dtype and
+ * the debug exports are ignored. */
+size_t sla2_backward_workspace_size(const sla2_desc* desc, float topk_frac);
+sla2_status sla2_backward(const sla2_desc* desc, const void* q, const void* k, const void* v, const float* proj_q,
+                          const float* proj_k, const float* alpha, float topk_frac, const float* dout, float* dq,
+                          float* dk, float* dv, float* dalpha, void* stream);
+
+/* The whole forward pass from HOST memory to HOST memory, with the copies
+ * overlapped with the computation. Heads are taken in groups of
+ * `heads_per_group` (per batch index, the last group of each batch index may
+ * be smaller): group g's Q, K and V are copied in on a library-owned stream
+ * while group g - 1 is computed on `stream` and group g - 2's output is copied
+ * out on another library-owned stream, through two device slots of the
+ * workspace. Each group is computed as sla2_forward_heads computes it, so the
+ * output is bit-identical to sla2_forward's for the same description.
+ *   q, k, v       : HOST bf16 [B][H][N][d]
+ *   proj_q, proj_k: HOST fp32 [H][d][d];  alpha: HOST fp32 [H][N/128]
+ *   out           : HOST bf16 or fp32 (desc->out_dtype) [B][H][N][d]
+ *   desc->workspace : DEVICE memory of sla2_forward_host_workspace_size bytes
+ *                   (the per-group forward workspace, the projections and
+ *                   alpha, and the two slots of group inputs and outputs)
+ *   1 <= heads_per_group <= H; desc's debug exports and stage_events must be
+ *   NULL (else SLA2_ERR_INVALID_ARG).
+ * Returns once everything is enqueued; out is complete when `stream` has
+ * reached that point (the call makes `stream` wait for the last copy out), and
+ * the host buffers must stay valid until then. Page-locked host memory lets
+ * the copies run asynchronously and concurrently; with pageable memory the
+ * result is the same but the copies serialise with the host. The copy streams
+ * and their events are created by the first call on each device and kept until
+ * the process exits; calls from several host threads are serialised while they
+ * enqueue. */
+size_t sla2_forward_host_workspace_size(const sla2_desc* desc, int heads_per_group, float topk_frac);
+sla2_status sla2_forward_host(const sla2_desc* desc, int heads_per_group, const void* q, const void* k,
+                              const void* v, const float* proj_q, const float* proj_k, const float* alpha,
+                              float topk_frac, void* out, void* stream);
 
 /* One rank's share of a head-sharded forward pass (the summary page's
  * future-work paragraph names multi-GPU execution; every step of the pass is

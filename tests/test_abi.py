@@ -151,3 +151,37 @@ def test_head_range_entry_point_rejects_bad_ranges_on_the_host(lib):
         assert lib.sla2_forward_heads(ctypes.byref(d), hb, hc, *args) == 1      # invalid argument
     d.dbg_scores = p                                                             # debug exports refused
     assert lib.sla2_forward_heads(ctypes.byref(d), 0, 2, *args) == 1
+
+
+def test_host_buffer_entry_point_rejects_bad_arguments_on_the_host(lib):
+    buf, p = _fake()
+    ws, pws = _fake()
+    d = _desc(H=4)
+    n2 = lib.sla2_forward_host_workspace_size(ctypes.byref(d), 2, 0.1)
+    n4 = lib.sla2_forward_host_workspace_size(ctypes.byref(d), 4, 0.1)
+    # the group's forward workspace plus two slots of group inputs and outputs
+    slot2 = 2 * 2 * (3 * 1024 * 64 * 2 + 1024 * 64 * 2)
+    assert n2 > lib.sla2_workspace_size_heads(ctypes.byref(d), 2, 0.1) + slot2
+    assert n4 > n2
+    for hpg in (0, -1, 5):
+        assert lib.sla2_forward_host_workspace_size(ctypes.byref(d), hpg, 0.1) == 0
+    args = [ctypes.c_void_p(p)] * 6 + [ctypes.c_float(0.1), ctypes.c_void_p(p + 4096), None]
+    d.workspace, d.workspace_bytes = pws, n2
+    for hpg in (0, 5):
+        assert lib.sla2_forward_host(ctypes.byref(d), hpg, *args) == 1          # invalid argument
+    d.workspace_bytes = n2 - 1
+    assert lib.sla2_forward_host(ctypes.byref(d), 2, *args) == 3                 # workspace too small
+    d.workspace_bytes = n2
+    d.stage_events = p                                                           # per-stage events refused
+    assert lib.sla2_forward_host(ctypes.byref(d), 2, *args) == 1
+    d.stage_events = None
+    bad = [None] + args[1:]
+    assert lib.sla2_forward_host(ctypes.byref(d), 2, *bad) == 1
+
+
+def test_host_binding_refuses_device_tensors_and_wrong_out():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sla2.forward_host(q, q, q, torch.zeros(1, 64, 64), torch.zeros(1, 64, 64), torch.zeros(1, 1), 0.5,
+                          torch.zeros(1, 1, 128, 32, dtype=torch.bfloat16))

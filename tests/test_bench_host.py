@@ -6,10 +6,10 @@ from oracle import sla2_oracle as O
 
 
 def test_launches_per_forward_follow_the_launch_sequence():
-    # pool, colmean, projections, logits, top-k, linear state, reduce, sparse, Z_i, epilogue
+    # pool, column means, projections, logits, top-k, linear state, reduce, sparse, epilogue
     w = WORKLOADS["wan1.3b"]
-    assert bench.launches_per_forward(w, O.topk_count(w.nk, w.topk_frac)) == 10
-    # every key block kept: no Z_i pass
+    assert bench.launches_per_forward(w, O.topk_count(w.nk, w.topk_frac)) == 9
+    # every key block kept: the same launches
     assert bench.launches_per_forward(w, w.nk) == 9
 
 

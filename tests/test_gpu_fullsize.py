@@ -8,7 +8,9 @@ the C ABI, against the CPU oracle on the same seeded inputs:
   k% = 100 with alpha = 1 against dense softmax attention (quantised and
   unquantised), and k% in {5, 10, 20} against the quantisation-emulating oracle;
 - one whole head of the headline workload (k% = 3, all 256 query blocks);
-- a head-sharded forward (sla2_forward_heads) reproducing the full call bit for bit.
+- a head-sharded forward (sla2_forward_heads) reproducing the full call bit for bit;
+- the host-buffer forward (sla2_forward_host, copies overlapped with the
+  computation head group by head group) reproducing the full call bit for bit.
 """
 import ctypes
 
@@ -238,3 +240,27 @@ def test_head_shards_reproduce_the_full_call_bit_for_bit(sla2, B, H, N, d, frac,
                                    hb, hc, out, quantize=quant)
         torch.cuda.synchronize()
         assert torch.equal(out, full), f"world {world}: sharded output differs"
+
+
+# ------------------------------------------------------------------ host buffers
+@pytest.mark.parametrize("B,H,N,d,frac,hpg,quant,f32", [(1, 12, 8192, 128, 0.03, 2, 1, False),
+                                                         (2, 5, 4096, 64, 0.1, 2, 1, True),
+                                                         (1, 3, 2048, 128, 0.1, 3, 0, False),
+                                                         (2, 3, 2048, 64, 0.2, 1, 1, False)])
+def test_host_buffer_forward_reproduces_the_device_call_bit_for_bit(sla2, B, H, N, d, frac, hpg, quant, f32):
+    """sla2_forward_host on page-locked host tensors (groups of `hpg` heads, the
+    last group of a batch index smaller where hpg does not divide H) writes into
+    host memory exactly what sla2_forward writes on the device."""
+    inp = make_custom(B, H, N, d, frac, seed=57)
+    dev = to_dev(inp)
+    dt = torch.float32 if f32 else torch.bfloat16
+    full = sla2.forward(dev["q"], dev["k"], dev["v"], dev["proj_q"], dev["proj_k"], dev["alpha"], frac,
+                        quantize=quant, out_dtype=dt)
+    host = {n: getattr(inp, n).contiguous().pin_memory() for n in ("q", "k", "v", "proj_q", "proj_k", "alpha")}
+    out = torch.full((B, H, N, d), float("nan"), dtype=dt).pin_memory()
+    for rep in range(2):   # a second call reuses the copy streams, events and workspace slots
+        out.fill_(float("nan"))
+        sla2.forward_host(host["q"], host["k"], host["v"], host["proj_q"], host["proj_k"], host["alpha"], frac, out,
+                          heads_per_group=hpg, quantize=quant)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(out, full.cpu()), f"call {rep}: host-buffer output differs"
