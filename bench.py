@@ -101,13 +101,16 @@ def work_model(w, k):
         "router_bytes": 2 * E * 3 + E,
         # linear state: read K, V (bf16), write K-hat, V-hat^T (8-bit), h_j^T tiles (fp16), z_j (fp32)
         "linear_bytes": 2 * E * 2 + 2 * E + BH * nk * d * d * 2 + BH * nk * d * 4,
-        # epilogue: read Q (bf16), O_s (fp32), h_j^T tiles once (fp16), write out (bf16); the
-        # repeated tile gather (k + 1 per query block) is L2 traffic, reported separately
-        "epilogue_bytes": 2 * E + 4 * E + 2 * E + BH * nk * d * d * 2,
-        "gather_bytes": BH * nq * (k + 1) * d * d * 2,   # per query block: H_total and the k selected h_j tiles
-        # epilogue MMAs as issued: phi(Q_i) (128 x d) times k + 1 tiles (d x d), fp16 in, fp32
-        # accumulate; the algorithmic work is one product phi(Q_i) H_i per query block
-        "epilogue_flops_issued": BH * nq * (k + 1) * 2 * 128 * d * d if k < nk else 0,
+        # linear apply + mix (selected-state product and epilogue): read Q (bf16), O_s (fp16
+        # on the quantised path), the h_j^T images once (fp16) and z_j, write out (bf16).
+        # The s H_i^T images the product hands to the epilogue (written, then read once) are
+        # an intermediate of this design, counted apart as hi_bytes.
+        "epilogue_bytes": (2 * E + 2 * E + BH * nk * d * d * 2 + BH * nk * d * 4 + 2 * E) if k < nk
+                          else 2 * E + 2 * E,
+        "hi_bytes": 2 * BH * nq * d * d * 2 if k < nk else 0,
+        # tensor work as issued: the dense mask product (nq x nk x d^2 per head; M is 0 / 1) and
+        # one phi(Q_i) (s H_i) per query block; the algorithmic work is the latter alone
+        "epilogue_flops_issued": (2 * BH * nq * nk * d * d + 2 * N * d * d * BH) if k < nk else 0,
         "epilogue_flops": 2 * N * d * d * BH if k < nk else 0,
     }
 
@@ -144,9 +147,9 @@ def measured_traffic(name):
 
 def launches_per_forward(w, k):
     """Kernels one forward launches: router 5 (pool, column means, both projections in
-    one launch, logits, top-k), linear state 2, sparse 1 and epilogue 1, whatever k."""
-    del w, k
-    return 5 + 2 + 1 + 1
+    one launch, logits, top-k), linear state 2, sparse 1, the selected-state product 1
+    and epilogue 1 (no selected-state product when every key block is selected)."""
+    return 5 + 2 + 1 + (2 if k < w.nk else 1)
 
 
 class ClockSampler:
@@ -495,12 +498,13 @@ def main():
             kern[n] = {"ms": msv, "bound": "tensor", "achieved": ach, "peak": p8, "unit": "TOPS", "frac": ach / p8,
                        "peak_source": p8_src}
         elif n == "epilogue":
-            # HBM-bound: read Q (bf16) and O_s (fp32), the h tiles once, write out; its
-            # tensor work is given beside it (algorithmic: one phi(Q_i) H_i per query block)
+            # HBM-bound: read Q, O_s, the h images once, write out; its tensor work is given
+            # beside it (algorithmic: one phi(Q_i) H_i per query block; issued: + the mask product)
             b = wm["epilogue_bytes"]
             ach = b / (msv * 1e-3) / 1e9
             kern[n] = {"ms": msv, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                        "algorithmic_bytes": b, "peak_source": f"{peak_src} HBM copy",
+                       "intermediate_bytes": wm["hi_bytes"],
                        "tensor_algorithmic_flops": wm["epilogue_flops"],
                        "tensor_issued_flops": wm["epilogue_flops_issued"],
                        "tensor_frac_algorithmic": wm["epilogue_flops"] / (msv * 1e-3) / 1e12 / p16,
@@ -538,7 +542,7 @@ def main():
         "roofline": roofline, "kernels": kern,
         "stages": "router = pass over Q/K/V + column means; linear_state = linear state + reduce on a second "
                   "stream, with the router's projections / logits / top-k concurrent on the caller's stream; "
-                  "sparse = sparse branch (Z_i concurrent); epilogue = linear apply + mix",
+                  "sparse = sparse branch; epilogue = selected-state product (s H_i, Z_i) + linear apply + mix",
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_forward(w, k) * K, "clocks": clk,
         "sparse_issued_tops": kern["sparse"]["achieved"],

@@ -54,8 +54,8 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 
 // Workspace regions (each 256-byte aligned).
 struct Layout {
-  size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart, zpart, Htot, Ztot,
-      htile, hscale, os, total;
+  size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, mask16, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart,
+      zpart, Htot, Ztot, htile, hscale, hi, Zi, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -78,6 +78,7 @@ Layout make_layout(const Shape& s, int quant) {
   L.scores = take(BH * nq * nk * 4);
   L.mask = take(BH * nq * nk);
   L.idx = take(BH * nq * k * 4);
+  L.mask16 = take(BH * nq * ((nk + 7) & ~size_t(7)) * 2);   // fp16 mask, rows padded to 8
   L.qhat = take(quant ? BH * N * d : 0);
   L.sq = take(BH * nq * 4);
   L.vamax = take(BH * d * 4);
@@ -93,6 +94,8 @@ Layout make_layout(const Shape& s, int quant) {
   L.Ztot = take(BH * d * 4);
   L.htile = take(BH * d * d * 2);    // fp16 s H_total^T operand tiles
   L.hscale = take(BH * 4);
+  L.hi = take(BH * nq * d * d * 2);  // fp16 s H_i^T operand images
+  L.Zi = take(BH * nq * d * 4);
   L.os = take(BH * N * d * (quant ? 2 : 4));   // fp16 O_s / s_v, or fp32 O_s
   L.total = off;
   return L;
@@ -211,12 +214,12 @@ sla2_status router_head(const sla2_desc* d, const Shape& s, const Layout& L, con
 
 // Router, second part: projections, logits and the hard top-k.
 sla2_status router_tail(const sla2_desc* d, const Shape& s, const Layout& L, const float* wq, const float* wk,
-                        uint8_t* mask, int32_t* idx, cudaStream_t st) {
+                        uint8_t* mask, int32_t* idx, cudaStream_t st, uint16_t* mask16 = nullptr) {
   SLA2_TRY(launch_proj(s, d->H, at<float>(d, L.qbar), at<float>(d, L.kbs), wq, wk, at<float>(d, L.A),
                        at<float>(d, L.Bk), st));
   float* scores = d->dbg_scores ? d->dbg_scores : at<float>(d, L.scores);
   SLA2_TRY(launch_scores(s, at<float>(d, L.A), at<float>(d, L.Bk), scores, st));
-  SLA2_TRY(launch_topk(s, scores, mask, idx, st));
+  SLA2_TRY(launch_topk(s, scores, mask, idx, st, mask16));
   return SLA2_OK;
 }
 
@@ -348,7 +351,8 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, o.vamax, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
                                 at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), aux->stream));
   SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
-  r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, st);
+  uint16_t* mask16 = s.k < s.nk ? at<uint16_t>(desc, L.mask16) : nullptr;
+  r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, st, mask16);
   if (r != SLA2_OK) return r;
   SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));   // join
   SLA2_TRY(mark(2));
@@ -377,14 +381,32 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   SLA2_TRY(launch_sparse(s, quant, tq, tk, tv, sa, st));
   SLA2_TRY(mark(3));
 
+  // the linear branch's s H_i^T and Z_i for every query block (one product with the mask)
+  if (s.k < s.nk) {
+    CUtensorMap tm, ti;
+    const uint64_t nk8 = ((uint64_t)s.nk + 7) & ~uint64_t(7);
+    if (!make_map(&tm, mask16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, nk8, (uint64_t)s.BH * s.nq, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&ti, at<void>(desc, L.h), CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)s.d * s.d,
+                  (uint64_t)s.BH * s.nk, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA2_ERR_CUDA;
+    HselArgs ha{};
+    ha.htile = at<uint16_t>(desc, L.htile);
+    ha.Ztot = at<float>(desc, L.Ztot);
+    ha.z = at<float>(desc, L.z);
+    ha.idx = idx;
+    ha.hi = at<uint16_t>(desc, L.hi);
+    ha.Zi = at<float>(desc, L.Zi);
+    ha.status = desc->status;
+    ha.budget_ns = g_budget_ns;
+    SLA2_TRY(launch_hsel(s, tm, ti, ha, st));
+  }
+
   EpilogueArgs ea{};
   ea.q = q;
-  ea.htile = at<uint16_t>(desc, L.htile);
-  ea.hT = at<uint16_t>(desc, L.h);
+  ea.hi = at<uint16_t>(desc, L.hi);
+  ea.Zi = at<float>(desc, L.Zi);
   ea.hscale = at<float>(desc, L.hscale);
-  ea.Ztot = at<float>(desc, L.Ztot);
-  ea.z = at<float>(desc, L.z);
-  ea.idx = idx;
   ea.os = os;
   ea.os_half = quant;
   ea.sv = at<float>(desc, L.sv);
@@ -396,7 +418,12 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  SLA2_TRY(launch_epilogue(s, ea, st));
+  CUtensorMap teq, tos;
+  if (!make_map(&teq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tos, quant ? os : q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, s.d, rows, 64, BQ,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return SLA2_ERR_CUDA;
+  SLA2_TRY(launch_epilogue(s, teq, tos, ea, st));
   SLA2_TRY(mark(4));
 
   // debug exports

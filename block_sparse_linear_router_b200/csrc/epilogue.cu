@@ -42,32 +42,42 @@ namespace sla2 {
 namespace {
 
 constexpr int EPI_COMPUTE = 256;          // warps 0-7
-constexpr int EPI_SUM_WARP0 = 8;          // warps 8-15
-constexpr int EPI_SUM = 256;
-constexpr int EPI_THREADS = EPI_COMPUTE + EPI_SUM;   // 16 warps: 128 registers a thread
+constexpr int EPI_LOAD_WARP = 8;          // warp 8: bulk copies of the s H_i^T images and Z_i
+constexpr int EPI_THREADS = EPI_COMPUTE + 32;
 
 template <int D>
 struct EpiCfg {
   static constexpr int SLABS = D / 64;               // K slabs of 64 fp16 (128 bytes)
   static constexpr int TILE = D * D * 2;             // one fp16 operand image (atom_off layout)
   static constexpr int SBO = SLABS * 1024;           // bytes between 8-row groups of an image
-  static constexpr int CHUNKS = TILE / 16;           // 16-byte chunks of an image
-  static constexpr int CPT = CHUNKS / EPI_SUM;       // chunks per sum thread (8 at d = 128, 2 at d = 64)
-  static constexpr int CPASS = CPT < 4 ? CPT : 4;    // chunks summed per pass (register budget)
   static constexpr int HC = D / 2;                   // features (and output columns) per compute thread
-  static constexpr int OFF_Z = 2 * TILE;                      // Z_i of two items [2][D]
-  static constexpr int OFF_XCH = OFF_Z + 2 * D * 4;           // row max per half [2][BQ]
+  static constexpr int RSLAB = BQ * 128;             // 128 rows x 64 16-bit columns, 128-byte swizzle
+  static constexpr int QB = SLABS * RSLAB;           // the item's Q rows (bf16)
+  static constexpr int OSB = SLABS * RSLAB;          // the item's O_s / s_v rows (fp16, quantised path)
+  static constexpr int ASLOT = TILE + QB;            // ring A: the s H_i^T image and the Q rows of an item
+  static constexpr int NA = 2;                       // ring A slots (freed when the item's MMA completes)
+  static constexpr int NO = D == 128 ? 2 : 4;        // ring O slots (freed after the item's readout)
+  static constexpr int OFF_O = NA * ASLOT;                    // ring O
+  static constexpr int OFF_Z = OFF_O + NO * OSB;              // Z_i [NA][D]
+  static constexpr int OFF_XCH = OFF_Z + NA * D * 4;          // row max per half [2][BQ]
   static constexpr int OFF_DEN = OFF_XCH + 2 * BQ * 4;        // denominator halves [2 buffers][2][BQ]
   static constexpr int OFF_BAR = OFF_DEN + 4 * BQ * 4;
-  static constexpr int NBAR = 11;
+  static constexpr int NBAR = 2 * NA + 2 * NO + 3;   // afull, afree [NA]; ofull, ofree [NO]; dfull [2]; drain
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
   static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
-  static_assert(TILE % 1024 == 0 && CHUNKS % EPI_SUM == 0 && CPT % CPASS == 0, "image buffers and chunk split");
+  static_assert(TILE % 1024 == 0 && ASLOT % 1024 == 0 && OFF_O % 1024 == 0 && OSB % 1024 == 0 && OFF_Z % 16 == 0,
+                "slot alignment (128-byte swizzle)");
   static constexpr int KSTEPS = D / 16;              // 16 fp16 (8 TMEM columns of A) per MMA
   static constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, D);   // fp16 x fp16 -> fp32, N = D
   static constexpr uint32_t ACOL = 2 * D;            // accumulators: columns b * D; A buffers: ACOL + b * D / 2
   static constexpr uint32_t TMEM_COLS = 512;
 };
+
+// Byte offset of logical 16-byte chunk `c` (8 16-bit columns) of row `r` in
+// rows staged by TMA as 64-column slabs with 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz_chunk(int r, int c) {
+  return (uint32_t)((c >> 3) * (BQ * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
 
 __device__ __forceinline__ void unpack8(const uint4& w, float (&x)[8]) {
   x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
@@ -81,17 +91,6 @@ __device__ __forceinline__ uint32_t h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// acc[0..7] += the eight fp16 values of a 16-byte chunk
-__device__ __forceinline__ void add_h8(float* acc, const uint4& w) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-    acc[2 * i] += f.x;
-    acc[2 * i + 1] += f.y;
-  }
-}
-
 // Read-only 16-byte load kept where it is written (its latency overlaps the
 // work in between instead of being moved down to the first use), with an L2
 // cache policy.
@@ -103,24 +102,8 @@ __device__ __forceinline__ uint4 ldg_v4_early(const uint4* p, uint64_t pol) {
   return r;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
-// Barriers over the 256 compute threads (id 1) and the 256 sum threads (id 2).
+// Barrier over the 256 compute threads (id 1).
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-__device__ __forceinline__ void sum_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
-__device__ __forceinline__ bool sum_sync_any(bool failed) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)failed)
-      : "memory");
-  return r != 0;
-}
-
 // Barrier over the 256 compute threads that also returns, to every one of
 // them, whether any of them passed `failed` (so all take the same exit).
 __device__ __forceinline__ bool compute_sync_any(bool failed) {
@@ -220,35 +203,40 @@ __device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, flo
 }
 
 template <int D>
-__global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, EpilogueArgs a) {
+__global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_constant__ CUtensorMap tq,
+                                                                  const __grid_constant__ CUtensorMap tos, Shape s,
+                                                                  EpilogueArgs a) {
   using C = EpiCfg<D>;
   extern __shared__ uint8_t esm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* hbuf = base;                   // [2] s H_i^T fp16 images
+  // ring A slot b: s H_i^T image at b * ASLOT, Q rows at + TILE; ring O slot c at OFF_O + c * OSB
   float* zbuf = reinterpret_cast<float*>(base + C::OFF_Z);
   float* xch = reinterpret_cast<float*>(base + C::OFF_XCH);
   float* den_s = reinterpret_cast<float*>(base + C::OFF_DEN);
-  uint64_t* hfull = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [2] H_i image and Z_i of an item written
-  uint64_t* hfree = hfull + 2;            // [2] the MMA reading image b has finished
-  uint64_t* dfull = hfull + 4;            // [2] accumulator complete
-  uint64_t* zfree = hfull + 6;            // [2] Z_i of an item used
-  uint64_t* zfull = hfull + 8;            // [2] Z_i of an item written
-  uint64_t* drain = hfull + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  int* abort_flag = reinterpret_cast<int*>(drain + 1) + 1;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [NA] image, Q rows and Z_i landed
+  uint64_t* afree = afull + C::NA;        // [NA] the item's MMA has completed (phi read Q before it)
+  uint64_t* ofull = afree + C::NA;        // [NO] O_s rows landed
+  uint64_t* ofree = ofull + C::NO;        // [NO] the item's readout is done
+  uint64_t* dfull = ofree + C::NO;        // [2] accumulator complete
+  uint64_t* drain = dfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + C::NBAR);
+  int* abort_flag = reinterpret_cast<int*>(afull + C::NBAR) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = s.BH * s.nq;
   const bool has_linear = s.k < s.nk;
 
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(hfull + b, 1);
-      mbar_init(hfree + b, 1);
-      mbar_init(zfree + b, EPI_COMPUTE);
-      mbar_init(zfull + b, 1);
-      mbar_init(dfull + b, 1);
+    for (int b = 0; b < C::NA; ++b) {
+      mbar_init(afull + b, 1);
+      mbar_init(afree + b, 1);
     }
+    for (int b = 0; b < C::NO; ++b) {
+      mbar_init(ofull + b, 1);
+      mbar_init(ofree + b, EPI_COMPUTE);
+    }
+    mbar_init(dfull, 1);
+    mbar_init(dfull + 1, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -262,67 +250,45 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= EPI_SUM_WARP0) {
-    // ---------------------------------------------------------------- sum warps
-    const int st = tid - EPI_SUM_WARP0 * 32;     // 0 .. 255
-    if (has_linear) {
-      const size_t tile_chunks = (size_t)C::CHUNKS;
-      const uint64_t keep = l2_policy_evict_last();   // an image is re-read by ~k query blocks of the head
-      bool ok = true;
+  if (warp == EPI_LOAD_WARP) {
+    // ---------------------------------------------------------------- loader
+    // lane 0, ring A: per item the s H_i^T image and the Z_i row (bulk copies) and the
+    //   Q rows (TMA, 64-column slabs), once the MMA of item it - NA has completed;
+    // lane 1, ring O: per item the fp16 O_s rows (TMA; quantised path only), once the
+    //   readout of item it - NO is done.
+    if (lane < 2 && has_linear && (lane == 0 || a.os_half)) {
+      const uint64_t once = l2_policy_evict_first();   // each is read once
+      const int NR = lane == 0 ? C::NA : C::NO;
+      uint64_t* rfull = lane == 0 ? afull : ofull;
+      uint64_t* rfree = lane == 0 ? afree : ofree;
       int it = 0;
+      bool ok = true;
       for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-        const int bh = w / s.nq, qi = w % s.nq;
-        const int b = it & 1;
-        const int32_t* sel = a.idx + ((size_t)bh * s.nq + qi) * s.k;
-        // the image and Z_i buffers b were last read for item it - 2
-        bool okw = true;
-        if (it >= 2) {
-          okw = mbar_wait(hfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns) &&
-                mbar_wait(zfree + b, ((it >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns);
+        const int sb = it % NR;
+        if (it >= NR && !mbar_wait(rfree + sb, ((it / NR) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
+          ok = false;
+          break;
         }
-        if (sum_sync_any(!okw)) { ok = false; break; }
-        // Z_i = Z_total - the selected z_j, in ascending block order
-        if (st < D) {
-          float acc = a.Ztot[(size_t)bh * D + st];
-          for (int n = 0; n < s.k; ++n) acc -= a.z[((size_t)bh * s.nk + __ldg(sel + n)) * D + st];
-          zbuf[b * D + st] = acc;
+        const int row0 = w * BQ;                   // (head, query block) w starts at row w * 128 of [BH*N]
+        if (lane == 0) {
+          uint8_t* slot = base + sb * C::ASLOT;
+          mbar_arrive_expect_tx(afull + sb, (uint32_t)(C::TILE + C::QB + D * 4));
+          bulk_load_hint(slot, a.hi + (size_t)w * D * D, (uint32_t)C::TILE, afull + sb, once);
+#pragma unroll
+          for (int sl = 0; sl < C::SLABS; ++sl)
+            tma_load_2d(slot + C::TILE + sl * C::RSLAB, &tq, afull + sb, sl * 64, row0);
+          bulk_load(zbuf + sb * D, a.Zi + (size_t)w * D, (uint32_t)(D * 4), afull + sb);
+        } else {
+          uint8_t* slot = base + C::OFF_O + sb * C::OSB;
+          mbar_arrive_expect_tx(ofull + sb, (uint32_t)C::OSB);
+#pragma unroll
+          for (int sl = 0; sl < C::SLABS; ++sl) tma_load_2d(slot + sl * C::RSLAB, &tos, ofull + sb, sl * 64, row0);
         }
-        sum_sync();
-        if (st == 0) mbar_arrive(zfull + b);
-        // s H_i^T = s H_total^T + sum of the selected -s h_j^T, chunk by chunk
-        const uint4* img0 = reinterpret_cast<const uint4*>(a.htile + (size_t)bh * D * D);
-        const uint4* imgs = reinterpret_cast<const uint4*>(a.hT);
-        uint4* dst = reinterpret_cast<uint4*>(hbuf + b * C::TILE);
-#pragma unroll 1
-        for (int pass = 0; pass < C::CPT / C::CPASS; ++pass) {
-          float acc[C::CPASS * 8];
-#pragma unroll
-          for (int c = 0; c < C::CPASS * 8; ++c) acc[c] = 0.f;
-          const int c0 = st + pass * C::CPASS * EPI_SUM;
-#pragma unroll
-          for (int c = 0; c < C::CPASS; ++c) add_h8(acc + c * 8, ldg_v4_early(img0 + c0 + c * EPI_SUM, keep));
-          int j_next = __ldg(sel);
-          for (int n = 0; n < s.k; ++n) {
-            const int j = j_next;
-            if (n + 1 < s.k) j_next = __ldg(sel + n + 1);
-            const uint4* img = imgs + ((size_t)bh * s.nk + j) * tile_chunks;
-            uint4 w4[C::CPASS];
-#pragma unroll
-            for (int c = 0; c < C::CPASS; ++c) w4[c] = ldg_v4_early(img + c0 + c * EPI_SUM, keep);
-#pragma unroll
-            for (int c = 0; c < C::CPASS; ++c) add_h8(acc + c * 8, w4[c]);
-          }
-#pragma unroll
-          for (int c = 0; c < C::CPASS; ++c)
-            dst[c0 + c * EPI_SUM] = make_uint4(h2(acc[c * 8], acc[c * 8 + 1]), h2(acc[c * 8 + 2], acc[c * 8 + 3]),
-                                               h2(acc[c * 8 + 4], acc[c * 8 + 5]), h2(acc[c * 8 + 6], acc[c * 8 + 7]));
-        }
-        fence_proxy_async_smem();
-        sum_sync();
-        if (st == 0) mbar_arrive(hfull + b);
       }
-      (void)ok;
+      if (!ok)   // copies in flight land before the CTA releases its shared memory
+        for (int q = it > NR ? it - NR : 0; q < it; ++q) mbar_wait_drain(rfull + q % NR, (q / NR) & 1, 20000000ull);
     }
+    __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warps
     constexpr int HC = C::HC;
@@ -352,93 +318,87 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         }
       }
     } else {
-      // readout of item `itp` (work index wp): 16 accumulator columns at a
-      // time scaled to O_l, mixed with O_s and stored; the accumulator is
-      // released after its last columns are read
+      // readout of item `itp` (work index wp): 16 accumulator columns at a time
+      // scaled to O_l, mixed with O_s (from the item's slot on the quantised path)
+      // and stored; then the slot is handed back to the loader
       auto readout = [&](int itp, int wp) -> bool {
         const int bh = wp / s.nq, qi = wp % s.nq;
         const float alpha = a.alpha[(size_t)(bh % a.H) * s.nq + qi];
         const float hsc = a.hscale[bh];
         const size_t row = row_of(wp);
         const int bp = itp & 1;
+        const int so = itp % C::NO;
+        const uint8_t* osl = base + C::OFF_O + so * C::OSB;
         const size_t off0 = row * D + fh * HC;
         OsChunk ch[2];
-        os_issue(a, off0, stream_pol, ch[0]);   // in flight during the wait
+        if (!a.os_half) os_issue(a, off0, stream_pol, ch[0]);   // fp32 O_s from global, in flight during the wait
         bool ok = mbar_wait(dfull + bp, (itp >> 1) & 1, abort_flag, a.status, a.budget_ns);
+        if (a.os_half) ok = ok && mbar_wait(ofull + so, (itp / C::NO) & 1, abort_flag, a.status, a.budget_ns);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         if (!ok) return false;
         const float inv = 1.f / (hsc * (den_s[(bp * 2) * BQ + r] + den_s[(bp * 2 + 1) * BQ + r]));
 #pragma unroll
         for (int cc = 0; cc < HC / 16; ++cc) {
-          if (cc + 1 < HC / 16) os_issue(a, off0 + (cc + 1) * 16, stream_pol, ch[(cc + 1) & 1]);
+          const int col = fh * HC + cc * 16;
+          if (a.os_half) {
+            ch[cc & 1].w[0] = *reinterpret_cast<const uint4*>(osl + swz_chunk(r, col / 8));
+            ch[cc & 1].w[1] = *reinterpret_cast<const uint4*>(osl + swz_chunk(r, col / 8 + 1));
+          } else if (cc + 1 < HC / 16) {
+            os_issue(a, off0 + (cc + 1) * 16, stream_pol, ch[(cc + 1) & 1]);
+          }
           uint32_t v[16];
-          tmem_ld16(tmem + lane_base + (uint32_t)(bp * D + fh * HC + cc * 16), v);
+          tmem_ld16(tmem + lane_base + (uint32_t)(bp * D + col), v);
           tmem_wait_ld();
           float osv[16];
-          os_convert<D>(a, bh, off0 + cc * 16, fh * HC + cc * 16, ch[cc & 1], osv);
+          os_convert<D>(a, bh, off0 + cc * 16, col, ch[cc & 1], osv);
           float ol[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) ol[c] = __uint_as_float(v[c]) * inv;
           mix_store<16>(a, off0 + cc * 16, alpha, osv, ol, stream_pol);
         }
         tc_fence_before();   // the reads are ordered before the next compute barrier (the MMA that reuses it)
+        mbar_arrive(ofree + so);
         return true;
       };
 
-      uint4 qv[HC / 8];                          // this thread's half row of Q (bf16)
-      auto load_q = [&](int w) {               // issued here, consumed one item later
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + row_of(w) * D + fh * HC);
-#pragma unroll
-        for (int i = 0; i < HC / 8; ++i) qv[i] = ldg_v4_early(src + i, stream_pol);
-      };
-      load_q(blockIdx.x);
       int it = 0, wprev = -1;
       bool ok = true, rd_ok = true, issued = false;
       for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-        const int bh = w / s.nq, qi = w % s.nq;
-        const int b = it & 1;
-        if (wprev >= 0) {                        // O_s of the previous item, read out below
-          const size_t esz = a.os_half ? 2 : 4;
-          const uint8_t* p = static_cast<const uint8_t*>(a.os) + (row_of(wprev) * D + fh * HC) * esz;
-          for (int c = 0; c < (int)(HC * esz); c += 128) prefetch_l2(p + c);
-        }
-        (void)bh;
-        (void)qi;
+        const int b = it & 1;                    // TMEM A buffer, accumulator and denominators
+        const int sb = it % C::NA;               // the item's ring A slot
+        const uint8_t* qs = base + sb * C::ASLOT + C::TILE;
+        bool fok = mbar_wait(afull + sb, (it / C::NA) & 1, abort_flag, a.status, a.budget_ns);
+        fok = __all_sync(0xffffffffu, fok);
+        ok = ok && fok;
         // ---- phi = softmax over the d features. Its normalisation cancels in
         // O_l = phi H_i / (phi Z_i), so the operand is e = exp(q - M) with M
         // the row max (exchanged between the two halves) and no row sum.
-        float m4[4];
-        {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int q = 0; q < HC / 8; ++q) {
           float v8[8];
-          unpack8(qv[0], v8);
-          m4[0] = fmaxf(v8[0], v8[4]); m4[1] = fmaxf(v8[1], v8[5]);
-          m4[2] = fmaxf(v8[2], v8[6]); m4[3] = fmaxf(v8[3], v8[7]);
+          unpack8(fok ? *reinterpret_cast<const uint4*>(qs + swz_chunk(r, fh * (HC / 8) + q)) : make_uint4(0u, 0u, 0u, 0u),
+                  v8);
 #pragma unroll
-          for (int q = 1; q < HC / 8; ++q) {
-            unpack8(qv[q], v8);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) m4[c & 3] = fmaxf(m4[c & 3], v8[c]);
-          }
+          for (int c = 0; c < 8; ++c) m4[c & 3] = fmaxf(m4[c & 3], v8[c]);
         }
         const float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         xch[fh * BQ + r] = m;
         compute_sync();
         const float mb = fmaxf(m, xch[(fh ^ 1) * BQ + r]) * kLog2e;
         // den = e . Z_i over this half of the features
-        bool zok = mbar_wait(zfull + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns);
-        zok = __all_sync(0xffffffffu, zok);
-        ok = ok && zok;
-        const float4* zi4 = reinterpret_cast<const float4*>(zbuf + b * D + fh * HC);
+        const float4* zi4 = reinterpret_cast<const float4*>(zbuf + sb * D + fh * HC);
         float d4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[HC / 2];
 #pragma unroll
         for (int q = 0; q < HC / 8; ++q) {
           float v8[8];
-          unpack8(qv[q], v8);
+          unpack8(fok ? *reinterpret_cast<const uint4*>(qs + swz_chunk(r, fh * (HC / 8) + q)) : make_uint4(0u, 0u, 0u, 0u),
+                  v8);
 #pragma unroll
           for (int c = 0; c < 8; c += 4) {
-            const float4 zz = zok ? zi4[(q * 8 + c) / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 zz = fok ? zi4[(q * 8 + c) / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
             const float p0 = ex2_approx(fmaf(v8[c], kLog2e, -mb)), p1 = ex2_approx(fmaf(v8[c + 1], kLog2e, -mb));
             const float p2 = ex2_approx(fmaf(v8[c + 2], kLog2e, -mb)), p3 = ex2_approx(fmaf(v8[c + 3], kLog2e, -mb));
             d4[0] = fmaf(p0, zz.x, d4[0]);
@@ -449,7 +409,6 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
             pk[(q * 8 + c) / 2 + 1] = h2(p2, p3);
           }
         }
-        mbar_arrive(zfree + b);
         den_s[(b * 2 + fh) * BQ + r] = (d4[0] + d4[1]) + (d4[2] + d4[3]);
         const uint32_t ta = tmem + lane_base + C::ACOL + (uint32_t)(b * (D / 2) + fh * (HC / 2));
         if constexpr (HC / 2 == 32) {
@@ -459,29 +418,20 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(Shape s, Epilo
         }
         tmem_wait_st();
         tc_fence_before();
-        {
-          const int wn = w + gridDim.x;          // the next item's Q rows, consumed next iteration
-          if (wn < total) load_q(wn);
-        }
         // every compute thread takes this exit together; past it, the phi operand is in
         // TMEM and the readout of item it - 2 (same accumulator) is complete
         if (compute_sync_any(!ok || !rd_ok)) { ok = false; break; }
-        if (tid == 0) {   // MMA issue: D_b = phi(Q_i) (s H_i) once the sum warps have written s H_i^T
+        if (tid == 0) {   // MMA issue: D_b = phi(Q_i) (s H_i), the image from the item's slot
           tc_fence_after();
-          if (mbar_wait(hfull + b, (it >> 1) & 1, abort_flag, a.status, a.budget_ns)) {
-            tc_fence_after();
-            const uint32_t acol = tmem + C::ACOL + (uint32_t)(b * (D / 2));
-            const uint64_t bd = make_sdesc(smem_u32(hbuf + b * C::TILE), C::SBO, LAYOUT_SW128);
+          const uint32_t acol = tmem + C::ACOL + (uint32_t)(b * (D / 2));
+          const uint64_t bd = make_sdesc(smem_u32(base + sb * C::ASLOT), C::SBO, LAYOUT_SW128);
 #pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ++ks)
-              mma_f16_ts(tmem + (uint32_t)(b * D), acol + ks * 8,
-                         bd + (uint64_t)(((ks >> 2) * 1024 + (ks & 3) * 32) >> 4), C::IDESC, ks != 0);
-            issued = true;
-            tc_commit(hfree + b);
-            tc_commit(dfull + b);
-          } else {
-            ok = false;     // seen by every compute thread at the next barrier; the readout's wait fails first
-          }
+          for (int ks = 0; ks < C::KSTEPS; ++ks)
+            mma_f16_ts(tmem + (uint32_t)(b * D), acol + ks * 8,
+                       bd + (uint64_t)(((ks >> 2) * 1024 + (ks & 3) * 32) >> 4), C::IDESC, ks != 0);
+          issued = true;
+          tc_commit(afree + sb);   // the image and the Q rows (read by phi before this) can be reloaded
+          tc_commit(dfull + b);
         }
         // ---- the previous item's readout overlaps this item's MMAs
         if (wprev >= 0) rd_ok = readout(it - 1, wprev);
@@ -506,17 +456,18 @@ constexpr int kSMs = 148;   // B200 streaming multiprocessors
 
 }  // namespace
 
-cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st) {
+cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const EpilogueArgs& a,
+                            cudaStream_t st) {
   const int total = s.BH * s.nq;
   const int grid = total < kSMs ? total : kSMs;
   if (s.d == 128) {
     auto k = epilogue_kernel<128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<128>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(tq, tos, s, a);
   } else {
     auto k = epilogue_kernel<64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<64>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(tq, tos, s, a);
   }
   return cudaGetLastError();
 }

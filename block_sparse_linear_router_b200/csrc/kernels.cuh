@@ -42,7 +42,10 @@ cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const float* k
 // logits s = A Bk^T / sqrt(d), fp32 [BH][nq][nk]
 cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float* scores, cudaStream_t st);
 // hard top-k per logit row (ties -> lower index), mask and ascending index list
-cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st);
+// mask16 (optional): the mask also as fp16 1 / 0 rows of nk8 = nk rounded up to 8
+// (zero padding), the A operand of the selected-state product (hsel.cu).
+cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st,
+                        uint16_t* mask16 = nullptr);
 int scores_topk_max_nk();
 // SoftTop-k relaxation of each logit row: sigmoid(P_c / tau + lambda), row sums k
 cudaError_t launch_soft_topk(const Shape& s, const float* scores, float tau, float* soft, float* lam,
@@ -97,14 +100,27 @@ cudaError_t launch_sparse(const Shape& s, int quant, const CUtensorMap& tq, cons
 size_t sparse_smem_bytes(int d, int quant);
 
 // ---- epilogue (epilogue.cu) -----------------------------------------------
-struct EpilogueArgs {
-  const void* q;          // bf16 [BH][N][d]
-  const uint16_t* htile;  // fp16 s H_total^T operand images [BH][d*d] (h_mode-2 layout)
-  const uint16_t* hT;     // fp16 -s h_j^T operand images [BH][nk][d*d] (h_mode 2)
-  const float* hscale;    // [BH] s
+// ---- selected-state product (hsel.cu) -----------------------------------------
+struct HselArgs {
+  const uint16_t* htile;  // fp16 s H_total^T operand images [BH][d*d]
   const float* Ztot;      // [BH][d] Z_total
   const float* z;         // [BH][nk][d] z_j
   const int32_t* idx;     // [BH][nq][k]
+  uint16_t* hi;           // out: fp16 s H_i^T operand images [BH][nq][d*d]
+  float* Zi;              // out: [BH][nq][d] Z_i
+  unsigned* status;
+  unsigned long long budget_ns;
+};
+// tmask: the fp16 mask [BH*nq][nk8], box {64, 128}; timg: the -s h_j^T images as a
+// [BH*nk][d*d] fp16 matrix, box {64, 64}; both with 128-byte swizzle.
+cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const HselArgs& a,
+                        cudaStream_t st);
+
+struct EpilogueArgs {
+  const void* q;          // bf16 [BH][N][d]
+  const uint16_t* hi;     // fp16 s H_i^T operand images [BH][nq][d*d]
+  const float* Zi;        // [BH][nq][d]
+  const float* hscale;    // [BH] s
   const void* os;         // [BH][N][d] O_s: fp32, or fp16 O_s / s_v when os_half
   int os_half;
   const float* sv;        // [BH][d] s_v (os_half)
@@ -117,7 +133,10 @@ struct EpilogueArgs {
   unsigned* status;
   unsigned long long budget_ns;
 };
-cudaError_t launch_epilogue(const Shape& s, const EpilogueArgs& a, cudaStream_t st);
+// tq: Q as [BH*N][d] bf16, box {64, 128}; tos: O_s as [BH*N][d] fp16, box {64, 128}
+// (used when os_half); both with 128-byte swizzle.
+cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const EpilogueArgs& a,
+                            cudaStream_t st);
 
 // ---- backward pass (backward.cu) ------------------------------------------
 struct BackwardArgs {

@@ -437,7 +437,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // that keeps every key above it and the lowest-indexed keys equal to it.
 __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ scores, int rows, int nk,
                                                                int k, uint8_t* __restrict__ mask,
-                                                               int32_t* __restrict__ idx) {
+                                                               int32_t* __restrict__ idx, uint16_t* __restrict__ mask16,
+                                                               int nk8) {
   extern __shared__ uint32_t keys_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * TOPK_WARPS + warp;
@@ -473,6 +474,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
     eq_seen += __popc(eqm);
     const uint32_t selm = __ballot_sync(0xffffffffu, sel);
     if (in) mask[(size_t)row * nk + j] = sel ? 1 : 0;
+    if (mask16 && j < nk8) mask16[(size_t)row * nk8 + j] = sel ? 0x3C00u : 0u;   // fp16 1 / 0, zero padding
     if (sel) idx[(size_t)row * k + pos + __popc(selm & lt)] = j;
     pos += __popc(selm);
   }
@@ -483,7 +485,8 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
 template <int NPL>
 __global__ void __launch_bounds__(TOPK_WARPS * 32, 1) topk_reg_kernel(const float* __restrict__ scores, int rows, int nk,
                                                                    int k, uint8_t* __restrict__ mask,
-                                                                   int32_t* __restrict__ idx) {
+                                                                   int32_t* __restrict__ idx,
+                                                                   uint16_t* __restrict__ mask16, int nk8) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * TOPK_WARPS + warp;
   if (row >= rows) return;
@@ -519,6 +522,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32, 1) topk_reg_kernel(const floa
     eq_seen += __popc(eqm);
     const uint32_t selm = __ballot_sync(0xffffffffu, sel);
     if (in) mask[(size_t)row * nk + j] = sel ? 1 : 0;
+    if (mask16 && j < nk8) mask16[(size_t)row * nk8 + j] = sel ? 0x3C00u : 0u;   // fp16 1 / 0, zero padding
     if (sel) idx[(size_t)row * k + pos + __popc(selm & lt)] = j;
     pos += __popc(selm);
   }
@@ -646,29 +650,31 @@ cudaError_t launch_scores(const Shape& s, const float* A, const float* Bk, float
 
 int scores_topk_max_nk() { return TOPK_MAX_NK; }
 
-cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st) {
+cudaError_t launch_topk(const Shape& s, const float* scores, uint8_t* mask, int32_t* idx, cudaStream_t st,
+                        uint16_t* mask16) {
+  const int nk8 = (s.nk + 7) & ~7;
   const int rows = s.BH * s.nq;
   const dim3 grid((rows + TOPK_WARPS - 1) / TOPK_WARPS), block(TOPK_WARPS * 32);
   if (s.nk <= 128) {
-    topk_reg_kernel<4><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    topk_reg_kernel<4><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx, mask16, nk8);
     return cudaGetLastError();
   }
   if (s.nk <= 256) {
-    topk_reg_kernel<8><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    topk_reg_kernel<8><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx, mask16, nk8);
     return cudaGetLastError();
   }
   if (s.nk <= 512) {
-    topk_reg_kernel<16><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    topk_reg_kernel<16><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx, mask16, nk8);
     return cudaGetLastError();
   }
   if (s.nk <= 1024) {
-    topk_reg_kernel<32><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx);
+    topk_reg_kernel<32><<<grid, block, 0, st>>>(scores, rows, s.nk, s.k, mask, idx, mask16, nk8);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)TOPK_WARPS * s.nk * sizeof(uint32_t);
   cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   topk_kernel<<<(rows + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, smem, st>>>(scores, rows, s.nk, s.k, mask,
-                                                                                   idx);
+                                                                                   idx, mask16, nk8);
   return cudaGetLastError();
 }
 

@@ -6,10 +6,11 @@ from oracle import sla2_oracle as O
 
 
 def test_launches_per_forward_follow_the_launch_sequence():
-    # pool, column means, projections, logits, top-k, linear state, reduce, sparse, epilogue
+    # pool, column means, projections, logits, top-k, linear state, reduce, sparse,
+    # selected-state product, epilogue
     w = WORKLOADS["wan1.3b"]
-    assert bench.launches_per_forward(w, O.topk_count(w.nk, w.topk_frac)) == 9
-    # every key block kept: the same launches
+    assert bench.launches_per_forward(w, O.topk_count(w.nk, w.topk_frac)) == 10
+    # every key block kept: no selected-state product
     assert bench.launches_per_forward(w, w.nk) == 9
 
 
