@@ -16,14 +16,18 @@
 //   Z_i     = Z_total - sum_{j selected} z_j     (fp32, ascending j, CUDA cores)
 // alongside it.
 //
-// One CTA per (128 query blocks, 256 image positions, head); 128 threads:
-// warp 0 lane 0 issues the TMA loads (A = M as fp16 [nq][nk8], K-major; B = the
-// images as a [nk][d*d] fp16 matrix, MN-major, 128-byte swizzle) into a
-// 2-stage ring, warp 1 lane 0 issues the tcgen05 kind::f16 MMAs (M = 128,
-// N = 256, fp32 accumulator in TMEM); then every thread reads one accumulator
-// row (a query block) back, adds s H_total^T, rounds and stores. Before that,
-// while the MMAs run, each thread forms Z_i for its query block on the
-// 256 / d features that belong to this CTA's image positions.
+// Persistent CTAs (one per SM) walk the tiles (head, 256 image positions, 128
+// query blocks; query-block tiles of the same positions on neighbouring CTAs, so
+// an image tile is fetched from HBM once and re-read from L2). 192 threads:
+//   warp 0    TMA producer: per tile and 64-key-block step, A = M as fp16
+//             [nq][nk8] (K-major) and B = the images as a [nk][d*d] fp16 matrix
+//             (MN-major, four 64-position slabs), 128-byte swizzle, into a
+//             4-stage ring that runs on across tiles;
+//   warp 1    MMA issuer: tcgen05 kind::f16, M = 128, N = 256, into one of two
+//             TMEM accumulators (the other one is being read out);
+//   warps 2-5 per tile: Z_i for the tile's query blocks on the 256 / d features
+//             that belong to its positions, then the accumulator row of their
+//             query block (one TMEM lane each) + s H_total^T, rounded and stored.
 #include <cuda_fp16.h>
 
 #include "device.cuh"
@@ -33,23 +37,23 @@ namespace sla2 {
 
 namespace {
 
-constexpr int HS_THREADS = 128;
-constexpr int HS_BM = 128;      // query blocks per tile
-constexpr int HS_BN = 256;      // image positions per tile
-constexpr int HS_BK = 64;       // key blocks per stage
-constexpr int HS_NST = 2;       // stages
+constexpr int HS_THREADS = 192;
+constexpr int HS_BM = 128;        // query blocks per tile
+constexpr int HS_BN = 256;        // image positions per tile
+constexpr int HS_BK = 64;         // key blocks per stage
+constexpr int HS_NST = 4;         // stages
 
 struct HsCfg {
   static constexpr int A_BYTES = HS_BM * HS_BK * 2;                // 16 KB, K-major, 128-byte rows
   static constexpr int SLAB = HS_BK * 128;                         // 64 key rows x 64 positions (8 KB)
   static constexpr int B_BYTES = (HS_BN / 64) * SLAB;              // 32 KB, MN-major, four slabs
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int OFF_HT = HS_NST * STAGE;                    // s H_total^T positions of the tile (fp32)
-  static constexpr int OFF_BAR = OFF_HT + HS_BN * 4;
-  static constexpr int SMEM = OFF_BAR + 8 * (2 * HS_NST + 2) + 16 + 1024;
+  static constexpr int OFF_BAR = HS_NST * STAGE;
+  static constexpr int NBAR = 2 * HS_NST + 4 + 1;                  // full, empty [NST]; tfull, tfree [2]; drain
+  static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
+  static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
   // fp16 x fp16 -> fp32, M = 128, N = 256, A K-major, B MN-major (bit 16)
   static constexpr uint32_t IDESC = make_idesc(1, 0, 0, HS_BM, HS_BN) | (1u << 16);
-  static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
 };
 
 __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
@@ -58,170 +62,205 @@ __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(HS_THREADS, 2) hsel_kernel(const __grid_constant__ CUtensorMap tmask,
+__global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_constant__ CUtensorMap tmask,
                                                              const __grid_constant__ CUtensorMap timg, Shape s,
                                                              HselArgs a) {
   using C = HsCfg;
-  constexpr int FPT = HS_BN / D;                 // Z features per CTA (2 at d = 128, 4 at d = 64)
+  constexpr int FPT = HS_BN / D;                 // Z features per position tile (2 at d = 128, 4 at d = 64)
+  constexpr int NT = D * D / HS_BN;              // position tiles per head
   extern __shared__ uint8_t hsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hsm_raw) + 1023) & ~uintptr_t(1023));
-  float* ht = reinterpret_cast<float*>(base + C::OFF_HT);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [NST]
   uint64_t* empty = full + HS_NST;                                    // [NST]
-  uint64_t* done = empty + HS_NST;
-  uint64_t* drain = done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  int* abort_flag = reinterpret_cast<int*>(drain + 1) + 1;
+  uint64_t* tfull = empty + HS_NST;                                   // [2] accumulator complete
+  uint64_t* tfree = tfull + 2;                                        // [2] accumulator read out
+  uint64_t* drain = tfree + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + C::NBAR);
+  int* abort_flag = reinterpret_cast<int*>(full + C::NBAR) + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * HS_BM, e0 = blockIdx.y * HS_BN, bh = blockIdx.z;
+  const int nmt = (s.nq + HS_BM - 1) / HS_BM;    // query-block tiles per head
+  const int tiles = s.BH * NT * nmt;
   const int nkt = (s.nk + HS_BK - 1) / HS_BK;
+  // tile t: query-block tile fastest, then position tile, then head
+  auto tile_of = [&](int t, int& bh, int& m0, int& e0) {
+    m0 = (t % nmt) * HS_BM;
+    e0 = ((t / nmt) % NT) * HS_BN;
+    bh = t / (nmt * NT);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < HS_NST; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull + i, 1);
+      mbar_init(tfree + i, 128);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, HS_BN);
+    tmem_alloc(tmem_slot, 2 * HS_BN);
     tmem_relinquish();
   }
-  // s H_total^T at this tile's positions, for the epilogue
-  for (int c = tid; c < HS_BN; c += HS_THREADS)
-    ht[c] = __half2float(__ushort_as_half(a.htile[(size_t)bh * D * D + e0 + c]));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  bool ok = true;
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int n = 0;
-      for (; n < nkt; ++n) {
-        const int st = n % HS_NST;
-        if (n >= HS_NST && !mbar_wait(empty + st, ((n / HS_NST) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sa = base + st * C::STAGE;
-        mbar_arrive_expect_tx(full + st, (uint32_t)C::STAGE);
-        tma_load_2d(sa, &tmask, full + st, n * HS_BK, bh * s.nq + m0);
+      uint32_t g = 0;   // stages filled, over all tiles
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        int bh, m0, e0;
+        tile_of(t, bh, m0, e0);
+        for (int n = 0; n < nkt; ++n, ++g) {
+          const int st = (int)(g % HS_NST);
+          if (g >= (uint32_t)HS_NST &&
+              !mbar_wait(empty + st, ((g / HS_NST) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = base + st * C::STAGE;
+          mbar_arrive_expect_tx(full + st, (uint32_t)C::STAGE);
+          tma_load_2d(sa, &tmask, full + st, n * HS_BK, bh * s.nq + m0);
 #pragma unroll
-        for (int sl = 0; sl < HS_BN / 64; ++sl)
-          tma_load_2d(sa + C::A_BYTES + sl * C::SLAB, &timg, full + st, e0 + sl * 64, bh * s.nk + n * HS_BK);
+          for (int sl = 0; sl < HS_BN / 64; ++sl)
+            tma_load_2d(sa + C::A_BYTES + sl * C::SLAB, &timg, full + st, e0 + sl * 64, bh * s.nk + n * HS_BK);
+        }
       }
       if (!ok)   // copies in flight land before the CTA releases its shared memory
-        for (int q = n > HS_NST ? n - HS_NST : 0; q < n; ++q)
+        for (uint32_t q = g > (uint32_t)HS_NST ? g - HS_NST : 0u; q < g; ++q)
           mbar_wait_drain(full + q % HS_NST, (q / HS_NST) & 1, 20000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool issued = false;
-      for (int n = 0; n < nkt; ++n) {
-        const int st = n % HS_NST;
-        if (!mbar_wait(full + st, (n / HS_NST) & 1, abort_flag, a.status, a.budget_ns)) {
+      uint32_t g = 0;
+      int i = 0;        // tiles of this CTA
+      bool ok = true, issued = false;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        if (i >= 2 && !mbar_wait(tfree + acc, ((i >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_u32(base + st * C::STAGE);
+        for (int n = 0; n < nkt; ++n, ++g) {
+          const int st = (int)(g % HS_NST);
+          if (!mbar_wait(full + st, (g / HS_NST) & 1, abort_flag, a.status, a.budget_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(base + st * C::STAGE);
 #pragma unroll
-        for (int ks = 0; ks < HS_BK / 16; ++ks) {
-          const uint64_t ad = make_sdesc(sa + ks * 32, 1024, LAYOUT_SW128);
-          const uint64_t bd = make_sdesc(sa + C::A_BYTES + ks * 2048, 1024, LAYOUT_SW128, C::SLAB);
-          mma_f16(tmem, ad, bd, C::IDESC, (n > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < HS_BK / 16; ++ks) {
+            const uint64_t ad = make_sdesc(sa + ks * 32, 1024, LAYOUT_SW128);
+            const uint64_t bd = make_sdesc(sa + C::A_BYTES + ks * 2048, 1024, LAYOUT_SW128, C::SLAB);
+            mma_f16(tmem + (uint32_t)(acc * HS_BN), ad, bd, C::IDESC, (n > 0 || ks > 0) ? 1u : 0u);
+          }
+          issued = true;
+          tc_commit(empty + st);
         }
-        issued = true;
-        tc_commit(empty + st);
+        if (ok) tc_commit(tfull + acc);
       }
-      if (ok) {
-        tc_commit(done);
-      } else if (issued) {   // issued MMAs finish before TMEM and shared memory are released
+      if (!ok && issued) {   // issued MMAs finish before TMEM and shared memory are released
         tc_commit(drain);
         mbar_wait_drain(drain, 0, 20000000ull);
       }
     }
-  }
-  __syncwarp();
-
-  // ------------------------------------------------------------ Z_i (overlaps the MMAs)
-  const int row = m0 + tid;                      // query block of this thread = TMEM lane
-  if (row < s.nq) {
-    const int f0 = blockIdx.y * FPT;
-    const int32_t* sel = a.idx + ((size_t)bh * s.nq + row) * s.k;
-    float zacc[FPT];
-#pragma unroll
-    for (int f = 0; f < FPT; ++f) zacc[f] = a.Ztot[(size_t)bh * D + f0 + f];
-    // eight selected blocks at a time: their indices, then their z slices, all in flight
-    // together; subtracted in ascending order
-    const float* zh = a.z + (size_t)bh * s.nk * D + f0;
-    for (int n0 = 0; n0 < s.k; n0 += 8) {
-      int jj[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) jj[u] = n0 + u < s.k ? __ldg(sel + n0 + u) : -1;
-      float zz[8][FPT];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int f = 0; f < FPT; ++f) zz[u][f] = jj[u] >= 0 ? __ldg(zh + (size_t)jj[u] * D + f) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (jj[u] >= 0)
-#pragma unroll
-          for (int f = 0; f < FPT; ++f) zacc[f] -= zz[u][f];
-    }
-#pragma unroll
-    for (int f = 0; f < FPT; ++f) a.Zi[((size_t)bh * s.nq + row) * D + f0 + f] = zacc[f];
-  }
-
-  // ------------------------------------------------------------ epilogue: s H_i^T = s H_total^T + G_i
-  bool dok = mbar_wait(done, 0, abort_flag, a.status, a.budget_ns);
-  dok = __all_sync(0xffffffffu, dok);
-  tc_fence_after();
-  if (dok) {
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    uint16_t* dst = a.hi + ((size_t)bh * s.nq + row) * D * D + e0;
-#pragma unroll 1
-    for (int cc = 0; cc < HS_BN / 32; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), v);
-      tmem_wait_ld();
+  } else {
+    // ------------------------------------------------------------ epilogue warps
+    const int qd = warp & 3;                     // TMEM lane quadrant
+    const int lr = qd * 32 + lane;               // accumulator row (query block within the tile)
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      int bh, m0, e0;
+      tile_of(t, bh, m0, e0);
+      const int row = m0 + lr;
+      const int acc = i & 1;
+      // Z_i = Z_total - the selected z_j (ascending j) on this position tile's features
       if (row < s.nq) {
+        const int f0 = (e0 / HS_BN) * FPT;
+        const int32_t* sel = a.idx + ((size_t)bh * s.nq + row) * s.k;
+        float zacc[FPT];
 #pragma unroll
-        for (int q = 0; q < 32; q += 8) {
-          const float* h = ht + cc * 32 + q;
-          *reinterpret_cast<uint4*>(dst + cc * 32 + q) =
-              make_uint4(h2u(h[0] + __uint_as_float(v[q]), h[1] + __uint_as_float(v[q + 1])),
-                         h2u(h[2] + __uint_as_float(v[q + 2]), h[3] + __uint_as_float(v[q + 3])),
-                         h2u(h[4] + __uint_as_float(v[q + 4]), h[5] + __uint_as_float(v[q + 5])),
-                         h2u(h[6] + __uint_as_float(v[q + 6]), h[7] + __uint_as_float(v[q + 7])));
+        for (int f = 0; f < FPT; ++f) zacc[f] = a.Ztot[(size_t)bh * D + f0 + f];
+        // eight selected blocks at a time: their indices, then their z slices, in flight together
+        const float* zh = a.z + (size_t)bh * s.nk * D + f0;
+        for (int n0 = 0; n0 < s.k; n0 += 8) {
+          int jj[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) jj[u] = n0 + u < s.k ? __ldg(sel + n0 + u) : -1;
+          float zz[8][FPT];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int f = 0; f < FPT; ++f) zz[u][f] = jj[u] >= 0 ? __ldg(zh + (size_t)jj[u] * D + f) : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (jj[u] >= 0)
+#pragma unroll
+              for (int f = 0; f < FPT; ++f) zacc[f] -= zz[u][f];
+        }
+#pragma unroll
+        for (int f = 0; f < FPT; ++f) a.Zi[((size_t)bh * s.nq + row) * D + f0 + f] = zacc[f];
+      }
+      // s H_i^T = s H_total^T + G_i at the tile's positions
+      bool ok = mbar_wait(tfull + acc, (i >> 1) & 1, abort_flag, a.status, a.budget_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (!ok) break;
+      const uint4* ht = reinterpret_cast<const uint4*>(a.htile + (size_t)bh * D * D + e0);
+      // kept in L2 for the epilogue, which reads every image once right after this kernel
+      const uint64_t keep = l2_policy_evict_last();
+      uint16_t* dst = a.hi + ((size_t)bh * s.nq + row) * D * D + e0;
+#pragma unroll 1
+      for (int cc = 0; cc < HS_BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + cc * 32), v);
+        tmem_wait_ld();
+        if (row < s.nq) {
+#pragma unroll
+          for (int q = 0; q < 32; q += 8) {
+            const uint4 hw = __ldg(ht + (cc * 32 + q) / 8);   // the same 16 bytes for every lane
+            const uint32_t hu[4] = {hw.x, hw.y, hw.z, hw.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hu[u]));
+              o[u] = h2u(h.x + __uint_as_float(v[q + 2 * u]), h.y + __uint_as_float(v[q + 2 * u + 1]));
+            }
+            stg_u4_policy(dst + cc * 32 + q, make_uint4(o[0], o[1], o[2], o[3]), keep);
+          }
         }
       }
+      tc_fence_before();
+      mbar_arrive(tfree + acc);   // the accumulator can take tile i + 2
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, HS_BN);
+    tmem_dealloc(tmem, 2 * HS_BN);
   }
 }
 
 }  // namespace
 
-size_t hsel_smem_bytes() { return (size_t)HsCfg::SMEM; }
-
 cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const HselArgs& a,
                         cudaStream_t st) {
-  const dim3 grid((s.nq + HS_BM - 1) / HS_BM, (s.d * s.d) / HS_BN, s.BH);
+  constexpr int kSMs = 148;   // B200 streaming multiprocessors
+  const int tiles = s.BH * ((s.d * s.d) / HS_BN) * ((s.nq + HS_BM - 1) / HS_BM);
+  const int grid = tiles < kSMs ? tiles : kSMs;
   if (s.d == 128) {
     cudaFuncSetAttribute(hsel_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, HsCfg::SMEM);
     hsel_kernel<128><<<grid, HS_THREADS, HsCfg::SMEM, st>>>(tmask, timg, s, a);
