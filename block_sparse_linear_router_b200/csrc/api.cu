@@ -418,12 +418,14 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   ea.ol_dbg = desc->dbg_ol;
   ea.status = desc->status;
   ea.budget_ns = g_budget_ns;
-  CUtensorMap teq, tos;
+  CUtensorMap teq, tos, tout;
   if (!make_map(&teq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tos, quant ? os : q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, s.d, rows, 64, BQ,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tout, desc->out_dtype ? q : out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, rows, 64, BQ,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return SLA2_ERR_CUDA;
-  SLA2_TRY(launch_epilogue(s, teq, tos, ea, st));
+  SLA2_TRY(launch_epilogue(s, teq, tos, tout, ea, st));
   SLA2_TRY(mark(4));
 
   // debug exports

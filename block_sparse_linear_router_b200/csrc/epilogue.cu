@@ -204,7 +204,8 @@ __device__ __forceinline__ void mix_store(const EpilogueArgs& a, size_t off, flo
 
 template <int D>
 __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_constant__ CUtensorMap tq,
-                                                                  const __grid_constant__ CUtensorMap tos, Shape s,
+                                                                  const __grid_constant__ CUtensorMap tos,
+                                                                  const __grid_constant__ CUtensorMap tout, Shape s,
                                                                   EpilogueArgs a) {
   using C = EpiCfg<D>;
   extern __shared__ uint8_t esm_raw[];
@@ -318,6 +319,9 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
         }
       }
     } else {
+      // bf16 output on the quantised path: staged in the O_s slot and stored by TMA
+      const bool tma_out = a.os_half && !a.out_f32;
+      int out_pending = -1;                      // thread 0: ring O slot whose TMA store may still read it
       // readout of item `itp` (work index wp): 16 accumulator columns at a time
       // scaled to O_l, mixed with O_s (from the item's slot on the quantised path)
       // and stored; then the slot is handed back to the loader
@@ -334,9 +338,9 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
         if (!a.os_half) os_issue(a, off0, stream_pol, ch[0]);   // fp32 O_s from global, in flight during the wait
         bool ok = mbar_wait(dfull + bp, (itp >> 1) & 1, abort_flag, a.status, a.budget_ns);
         if (a.os_half) ok = ok && mbar_wait(ofull + so, (itp / C::NO) & 1, abort_flag, a.status, a.budget_ns);
-        ok = __all_sync(0xffffffffu, ok);
+        // every compute thread takes the same exit (the output path below has a barrier)
+        if (compute_sync_any(!ok)) return false;
         tc_fence_after();
-        if (!ok) return false;
         const float inv = 1.f / (hsc * (den_s[(bp * 2) * BQ + r] + den_s[(bp * 2 + 1) * BQ + r]));
 #pragma unroll
         for (int cc = 0; cc < HC / 16; ++cc) {
@@ -355,10 +359,46 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
           float ol[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) ol[c] = __uint_as_float(v[c]) * inv;
-          mix_store<16>(a, off0 + cc * 16, alpha, osv, ol, stream_pol);
+          if (tma_out) {
+            float o[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) o[c] = alpha * osv[c] + (1.f - alpha) * ol[c];
+            uint8_t* ow = const_cast<uint8_t*>(osl);
+            *reinterpret_cast<uint4*>(ow + swz_chunk(r, col / 8)) =
+                make_uint4(cvt_bf16x2(o[0], o[1]), cvt_bf16x2(o[2], o[3]), cvt_bf16x2(o[4], o[5]), cvt_bf16x2(o[6], o[7]));
+            *reinterpret_cast<uint4*>(ow + swz_chunk(r, col / 8 + 1)) =
+                make_uint4(cvt_bf16x2(o[8], o[9]), cvt_bf16x2(o[10], o[11]), cvt_bf16x2(o[12], o[13]),
+                           cvt_bf16x2(o[14], o[15]));
+            if (a.ol_dbg) {
+#pragma unroll
+              for (int c = 0; c < 16; c += 4)
+                *reinterpret_cast<float4*>(a.ol_dbg + off0 + cc * 16 + c) = make_float4(ol[c], ol[c + 1], ol[c + 2], ol[c + 3]);
+            }
+          } else {
+            mix_store<16>(a, off0 + cc * 16, alpha, osv, ol, stream_pol);
+          }
         }
         tc_fence_before();   // the reads are ordered before the next compute barrier (the MMA that reuses it)
-        mbar_arrive(ofree + so);
+        if (tma_out) {
+          // the bf16 rows are in the O_s slot (each thread overwrote the chunks it read):
+          // thread 0 stores them with TMA and releases the slot once the store has read it
+          fence_proxy_async_smem();
+          compute_sync();
+          if (tid == 0) {
+            if (out_pending >= 0) {
+              bulk_wait_read0();
+              mbar_arrive(ofree + out_pending);
+            }
+#pragma unroll
+            for (int sl = 0; sl < C::SLABS; ++sl) tma_store_2d(&tout, osl + sl * C::RSLAB, sl * 64, wp * BQ);
+            bulk_commit();
+            out_pending = so;
+          } else {
+            mbar_arrive(ofree + so);
+          }
+        } else {
+          mbar_arrive(ofree + so);
+        }
         return true;
       };
 
@@ -438,6 +478,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
         wprev = w;
       }
       if (ok && rd_ok && wprev >= 0) rd_ok = readout(it - 1, wprev);
+      if (tid == 0 && out_pending >= 0) bulk_wait0();   // the last output rows have reached global memory
       if (tid == 0 && issued && !(ok && rd_ok)) {   // issued MMAs finish before TMEM and shared memory are released
         tc_commit(drain);
         mbar_wait_drain(drain, 0, 20000000ull);
@@ -456,18 +497,18 @@ constexpr int kSMs = 148;   // B200 streaming multiprocessors
 
 }  // namespace
 
-cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const EpilogueArgs& a,
-                            cudaStream_t st) {
+cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const CUtensorMap& tout,
+                            const EpilogueArgs& a, cudaStream_t st) {
   const int total = s.BH * s.nq;
   const int grid = total < kSMs ? total : kSMs;
   if (s.d == 128) {
     auto k = epilogue_kernel<128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<128>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(tq, tos, s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<128>::SMEM, st>>>(tq, tos, tout, s, a);
   } else {
     auto k = epilogue_kernel<64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, EpiCfg<64>::SMEM);
-    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(tq, tos, s, a);
+    k<<<grid, EPI_THREADS, EpiCfg<64>::SMEM, st>>>(tq, tos, tout, s, a);
   }
   return cudaGetLastError();
 }

@@ -48,7 +48,8 @@ struct HsCfg {
   static constexpr int SLAB = HS_BK * 128;                         // 64 key rows x 64 positions (8 KB)
   static constexpr int B_BYTES = (HS_BN / 64) * SLAB;              // 32 KB, MN-major, four slabs
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int OFF_BAR = HS_NST * STAGE;
+  static constexpr int OFF_STG = HS_NST * STAGE;                  // output staging, 4 warps x 32 rows x 128 B
+  static constexpr int OFF_BAR = OFF_STG + 4 * 32 * 128;
   static constexpr int NBAR = 2 * HS_NST + 4 + 1;                  // full, empty [NST]; tfull, tfree [2]; drain
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
   static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
@@ -221,25 +222,40 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
       const uint4* ht = reinterpret_cast<const uint4*>(a.htile + (size_t)bh * D * D + e0);
       // kept in L2 for the epilogue, which reads every image once right after this kernel
       const uint64_t keep = l2_policy_evict_last();
-      uint16_t* dst = a.hi + ((size_t)bh * s.nq + row) * D * D + e0;
+      // 64 positions at a time: each lane converts its row's 128 bytes into the warp's
+      // staging rows (16-byte chunk k of row r at chunk k ^ (r & 7): conflict-free both
+      // ways), then the warp stores 4 whole rows' 128 bytes per instruction
+      uint8_t* stg = base + C::OFF_STG + (qd * 32) * 128;
 #pragma unroll 1
-      for (int cc = 0; cc < HS_BN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + cc * 32), v);
+      for (int c64 = 0; c64 < HS_BN / 64; ++c64) {
+        uint4 hv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) hv[k] = __ldg(ht + c64 * 8 + k);   // the same 16 bytes for every lane
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + c64 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + c64 * 64 + 32),
+                  *reinterpret_cast<uint32_t(*)[32]>(v + 32));
         tmem_wait_ld();
-        if (row < s.nq) {
+        __syncwarp();   // the previous chunk's staging rows have been read
 #pragma unroll
-          for (int q = 0; q < 32; q += 8) {
-            const uint4 hw = __ldg(ht + (cc * 32 + q) / 8);   // the same 16 bytes for every lane
-            const uint32_t hu[4] = {hw.x, hw.y, hw.z, hw.w};
-            uint32_t o[4];
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t hu[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+          uint32_t o[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hu[u]));
-              o[u] = h2u(h.x + __uint_as_float(v[q + 2 * u]), h.y + __uint_as_float(v[q + 2 * u + 1]));
-            }
-            stg_u4_policy(dst + cc * 32 + q, make_uint4(o[0], o[1], o[2], o[3]), keep);
+          for (int u = 0; u < 4; ++u) {
+            const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hu[u]));
+            o[u] = h2u(h.x + __uint_as_float(v[k * 8 + 2 * u]), h.y + __uint_as_float(v[k * 8 + 2 * u + 1]));
           }
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = i * 4 + (lane >> 3), k = lane & 7;   // warp row, 16-byte chunk
+          const int grow = m0 + qd * 32 + rr;
+          const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((k ^ (rr & 7)) << 4));
+          if (grow < s.nq)
+            stg_u4_policy(a.hi + ((size_t)bh * s.nq + grow) * D * D + e0 + c64 * 64 + k * 8, val, keep);
         }
       }
       tc_fence_before();

@@ -134,9 +134,10 @@ struct EpilogueArgs {
   unsigned long long budget_ns;
 };
 // tq: Q as [BH*N][d] bf16, box {64, 128}; tos: O_s as [BH*N][d] fp16, box {64, 128}
-// (used when os_half); both with 128-byte swizzle.
-cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const EpilogueArgs& a,
-                            cudaStream_t st);
+// (used when os_half); tout: out as [BH*N][d] bf16, box {64, 128} (used when os_half
+// and the output is bf16); all with 128-byte swizzle.
+cudaError_t launch_epilogue(const Shape& s, const CUtensorMap& tq, const CUtensorMap& tos, const CUtensorMap& tout,
+                            const EpilogueArgs& a, cudaStream_t st);
 
 // ---- backward pass (backward.cu) ------------------------------------------
 struct BackwardArgs {
