@@ -116,7 +116,8 @@ def work_model(w, k):
 
 
 # DRAM bytes per launch measured by ncu (summaries under profiles/), valid only for the
-# kernel source they were taken on: sha256 prefix of the kernel file + device.cuh + kernels.cuh.
+# kernel source they were taken on: sha256 prefix of the stage's kernel file(s) ("a.cu+b.cu")
+# + device.cuh + kernels.cuh.
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum, --set full capture
     "sparse": ("sparse.cu", "3a73ccef7b0d189c", 298.1e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
@@ -137,7 +138,7 @@ def measured_traffic(name):
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_linear_router_b200", "csrc")
     h = hashlib.sha256()
     try:
-        for part in (f, "device.cuh", "kernels.cuh"):
+        for part in tuple(f.split("+")) + ("device.cuh", "kernels.cuh"):
             with open(os.path.join(csrc, part), "rb") as fh:
                 h.update(fh.read())
     except OSError:

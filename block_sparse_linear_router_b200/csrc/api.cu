@@ -55,7 +55,7 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 // Workspace regions (each 256-byte aligned).
 struct Layout {
   size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, mask16, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart,
-      zpart, Htot, Ztot, htile, hscale, hi, Zi, os, total;
+      zpart, Htot, Ztot, htile, hscale, hi, Zi, z16, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -88,6 +88,7 @@ Layout make_layout(const Shape& s, int quant) {
   L.sv = take(BH * d * 4);
   L.h = take(BH * nk * d * d * 2);   // fp16 -s h_j^T operand tiles
   L.z = take(BH * nk * d * 4);
+  L.z16 = take(BH * nk * d * 2);     // fp16 z_j, the selected-state product's operand
   L.hpart = take(BH * G * d * d * 4);
   L.zpart = take(BH * G * d * 4);
   L.Htot = take(BH * d * d * 4);
@@ -349,7 +350,8 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   o.budget_ns = g_budget_ns;
   SLA2_TRY(launch_linear_state(s, k, v, at<float>(desc, L.c32), o, aux->stream));
   SLA2_TRY(launch_linear_reduce(s, o.hpart, o.zpart, o.vamax, at<float>(desc, L.Htot), at<float>(desc, L.Ztot),
-                                at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), aux->stream));
+                                at<uint16_t>(desc, L.htile), at<float>(desc, L.hscale), aux->stream, o.z,
+                                at<uint16_t>(desc, L.z16)));
   SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
   uint16_t* mask16 = s.k < s.nk ? at<uint16_t>(desc, L.mask16) : nullptr;
   r = router_tail(desc, s, L, proj_q, proj_k, mask, idx, st, mask16);
@@ -383,23 +385,23 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
 
   // the linear branch's s H_i^T and Z_i for every query block (one product with the mask)
   if (s.k < s.nk) {
-    CUtensorMap tm, ti;
+    CUtensorMap tm, ti, tz;
     const uint64_t nk8 = ((uint64_t)s.nk + 7) & ~uint64_t(7);
     if (!make_map(&tm, mask16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, nk8, (uint64_t)s.BH * s.nq, 64, 128,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&ti, at<void>(desc, L.h), CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)s.d * s.d,
+                  (uint64_t)s.BH * s.nk, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tz, at<void>(desc, L.z16), CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)s.d,
                   (uint64_t)s.BH * s.nk, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return SLA2_ERR_CUDA;
     HselArgs ha{};
     ha.htile = at<uint16_t>(desc, L.htile);
     ha.Ztot = at<float>(desc, L.Ztot);
-    ha.z = at<float>(desc, L.z);
-    ha.idx = idx;
     ha.hi = at<uint16_t>(desc, L.hi);
     ha.Zi = at<float>(desc, L.Zi);
     ha.status = desc->status;
     ha.budget_ns = g_budget_ns;
-    SLA2_TRY(launch_hsel(s, tm, ti, ha, st));
+    SLA2_TRY(launch_hsel(s, tm, ti, tz, ha, st));
   }
 
   EpilogueArgs ea{};

@@ -42,7 +42,7 @@ namespace sla2 {
 namespace {
 
 constexpr int EPI_COMPUTE = 256;          // warps 0-7
-constexpr int EPI_LOAD_WARP = 8;          // warp 8: bulk copies of the s H_i^T images and Z_i
+constexpr int EPI_LOAD_WARP = 8;          // warp 8: bulk copies of the s H_i^T images and Z_i, Q and O_s rows
 constexpr int EPI_THREADS = EPI_COMPUTE + 32;
 
 template <int D>

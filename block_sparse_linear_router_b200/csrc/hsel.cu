@@ -1,7 +1,7 @@
 // The linear branch's per-query-block state (SLA2 summary page, step 3:
-// H_i = H_total - sum of the selected h_j, Z_i likewise; SLA2 detail page §7
-// note 2: the h_j are precomputed per key block and accumulated per query
-// block), for every (head, query block) at once.
+// H_i = H_total - sum of the selected h_j; SLA2 detail page §7 note 2: the h_j
+// are precomputed per key block and accumulated per query block), for every
+// (head, query block) at once.
 //
 // The selected blocks' share is a product with the router's block mask M
 // (nq x nk, 0 / 1): G = M S, where row j of S is the linear-state pass's fp16
@@ -12,9 +12,9 @@
 // reads each image once per 128 query blocks, and its 2 * nq * nk * d^2 flops
 // take a few tens of microseconds. Then
 //   s H_i^T = s H_total^T + G_i          (fp32 accumulation, rounded once to fp16)
-// is written in the same operand layout, and
-//   Z_i     = Z_total - sum_{j selected} z_j     (fp32, ascending j, CUDA cores)
-// alongside it.
+// is written in the same operand layout, where the epilogue reads it. The same
+// product with the fp16 z_j as rows gives Z_i = Z_total - sum of the selected z_j
+// (one more tile of N = d per 128 query blocks, written as fp32).
 //
 // Persistent CTAs (one per SM) walk the tiles (head, 256 image positions, 128
 // query blocks; query-block tiles of the same positions on neighbouring CTAs, so
@@ -25,9 +25,9 @@
 //             4-stage ring that runs on across tiles;
 //   warp 1    MMA issuer: tcgen05 kind::f16, M = 128, N = 256, into one of two
 //             TMEM accumulators (the other one is being read out);
-//   warps 2-5 per tile: Z_i for the tile's query blocks on the 256 / d features
-//             that belong to its positions, then the accumulator row of their
-//             query block (one TMEM lane each) + s H_total^T, rounded and stored.
+//   warps 2-5 per tile: the tile's s H_total^T positions into shared memory,
+//             then the accumulator row of their query block (one TMEM lane
+//             each) + s H_total^T, rounded and stored through per-warp staging.
 #include <cuda_fp16.h>
 
 #include "device.cuh"
@@ -49,12 +49,16 @@ struct HsCfg {
   static constexpr int B_BYTES = (HS_BN / 64) * SLAB;              // 32 KB, MN-major, four slabs
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int OFF_STG = HS_NST * STAGE;                  // output staging, 4 warps x 32 rows x 128 B
-  static constexpr int OFF_BAR = OFF_STG + 4 * 32 * 128;
+  static constexpr int OFF_HT = OFF_STG + 4 * 32 * 128;           // s H_total^T at the tile's positions (fp32)
+  static constexpr int OFF_BAR = OFF_HT + HS_BN * 4;
   static constexpr int NBAR = 2 * HS_NST + 4 + 1;                  // full, empty [NST]; tfull, tfree [2]; drain
   static constexpr int SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
   static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
-  // fp16 x fp16 -> fp32, M = 128, N = 256, A K-major, B MN-major (bit 16)
+  // fp16 x fp16 -> fp32, M = 128, N = 256 (image tiles) or d (the z tile), A K-major,
+  // B MN-major (bit 16)
   static constexpr uint32_t IDESC = make_idesc(1, 0, 0, HS_BM, HS_BN) | (1u << 16);
+  static constexpr uint32_t IDESC_Z128 = make_idesc(1, 0, 0, HS_BM, 128) | (1u << 16);
+  static constexpr uint32_t IDESC_Z64 = make_idesc(1, 0, 0, HS_BM, 64) | (1u << 16);
 };
 
 __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
@@ -64,11 +68,11 @@ __device__ __forceinline__ uint32_t h2u(float lo, float hi) {
 
 template <int D>
 __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_constant__ CUtensorMap tmask,
-                                                             const __grid_constant__ CUtensorMap timg, Shape s,
+                                                             const __grid_constant__ CUtensorMap timg,
+                                                             const __grid_constant__ CUtensorMap tz, Shape s,
                                                              HselArgs a) {
   using C = HsCfg;
-  constexpr int FPT = HS_BN / D;                 // Z features per position tile (2 at d = 128, 4 at d = 64)
-  constexpr int NT = D * D / HS_BN;              // position tiles per head
+  constexpr int NT = D * D / HS_BN + 1;          // position tiles per head, the last one z
   extern __shared__ uint8_t hsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hsm_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [NST]
@@ -128,11 +132,18 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
             break;
           }
           uint8_t* sa = base + st * C::STAGE;
-          mbar_arrive_expect_tx(full + st, (uint32_t)C::STAGE);
+          const bool zt = e0 == (NT - 1) * HS_BN;   // the z tile: D columns of z_j
+          mbar_arrive_expect_tx(full + st, (uint32_t)(C::A_BYTES + (zt ? (D / 64) * C::SLAB : C::B_BYTES)));
           tma_load_2d(sa, &tmask, full + st, n * HS_BK, bh * s.nq + m0);
+          if (zt) {
 #pragma unroll
-          for (int sl = 0; sl < HS_BN / 64; ++sl)
-            tma_load_2d(sa + C::A_BYTES + sl * C::SLAB, &timg, full + st, e0 + sl * 64, bh * s.nk + n * HS_BK);
+            for (int sl = 0; sl < D / 64; ++sl)
+              tma_load_2d(sa + C::A_BYTES + sl * C::SLAB, &tz, full + st, sl * 64, bh * s.nk + n * HS_BK);
+          } else {
+#pragma unroll
+            for (int sl = 0; sl < HS_BN / 64; ++sl)
+              tma_load_2d(sa + C::A_BYTES + sl * C::SLAB, &timg, full + st, e0 + sl * 64, bh * s.nk + n * HS_BK);
+          }
         }
       }
       if (!ok)   // copies in flight land before the CTA releases its shared memory
@@ -147,6 +158,8 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
       bool ok = true, issued = false;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
         const int acc = i & 1;
+        const bool zt = (t / nmt) % NT == NT - 1;
+        const uint32_t idesc = zt ? (D == 128 ? C::IDESC_Z128 : C::IDESC_Z64) : C::IDESC;
         if (i >= 2 && !mbar_wait(tfree + acc, ((i >> 1) - 1) & 1, abort_flag, a.status, a.budget_ns)) {
           ok = false;
           break;
@@ -164,7 +177,7 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
           for (int ks = 0; ks < HS_BK / 16; ++ks) {
             const uint64_t ad = make_sdesc(sa + ks * 32, 1024, LAYOUT_SW128);
             const uint64_t bd = make_sdesc(sa + C::A_BYTES + ks * 2048, 1024, LAYOUT_SW128, C::SLAB);
-            mma_f16(tmem + (uint32_t)(acc * HS_BN), ad, bd, C::IDESC, (n > 0 || ks > 0) ? 1u : 0u);
+            mma_f16(tmem + (uint32_t)(acc * HS_BN), ad, bd, idesc, (n > 0 || ks > 0) ? 1u : 0u);
           }
           issued = true;
           tc_commit(empty + st);
@@ -185,41 +198,51 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       int bh, m0, e0;
       tile_of(t, bh, m0, e0);
-      const int row = m0 + lr;
       const int acc = i & 1;
-      // Z_i = Z_total - the selected z_j (ascending j) on this position tile's features
-      if (row < s.nq) {
-        const int f0 = (e0 / HS_BN) * FPT;
-        const int32_t* sel = a.idx + ((size_t)bh * s.nq + row) * s.k;
-        float zacc[FPT];
+      if (e0 == (NT - 1) * HS_BN) {
+        // the z tile: Z_i = Z_total - G_i, fp32, one query block per thread
+        bool ok = mbar_wait(tfull + acc, (i >> 1) & 1, abort_flag, a.status, a.budget_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (!ok) break;
+        const int row = m0 + lr;
+        const float* zt = a.Ztot + (size_t)bh * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + cc * 32), v);
+          tmem_wait_ld();
+          if (row < s.nq) {
+            float* dst = a.Zi + ((size_t)bh * s.nq + row) * D + cc * 32;
 #pragma unroll
-        for (int f = 0; f < FPT; ++f) zacc[f] = a.Ztot[(size_t)bh * D + f0 + f];
-        // eight selected blocks at a time: their indices, then their z slices, in flight together
-        const float* zh = a.z + (size_t)bh * s.nk * D + f0;
-        for (int n0 = 0; n0 < s.k; n0 += 8) {
-          int jj[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) jj[u] = n0 + u < s.k ? __ldg(sel + n0 + u) : -1;
-          float zz[8][FPT];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-#pragma unroll
-            for (int f = 0; f < FPT; ++f) zz[u][f] = jj[u] >= 0 ? __ldg(zh + (size_t)jj[u] * D + f) : 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (jj[u] >= 0)
-#pragma unroll
-              for (int f = 0; f < FPT; ++f) zacc[f] -= zz[u][f];
+            for (int c = 0; c < 32; c += 4) {
+              const float4 zz = __ldg(reinterpret_cast<const float4*>(zt + cc * 32 + c));
+              *reinterpret_cast<float4*>(dst + c) =
+                  make_float4(zz.x - __uint_as_float(v[c]), zz.y - __uint_as_float(v[c + 1]),
+                              zz.z - __uint_as_float(v[c + 2]), zz.w - __uint_as_float(v[c + 3]));
+            }
+          }
         }
-#pragma unroll
-        for (int f = 0; f < FPT; ++f) a.Zi[((size_t)bh * s.nq + row) * D + f0 + f] = zacc[f];
+        tc_fence_before();
+        mbar_arrive(tfree + acc);
+        continue;
+      }
+      // the tile's s H_total^T positions (fp32) into shared memory, two per thread; the
+      // previous tile's readers are past the barrier that ended it
+      float* hts = reinterpret_cast<float*>(base + C::OFF_HT);
+      {
+        const uint32_t hw = __ldg(reinterpret_cast<const uint32_t*>(a.htile + (size_t)bh * D * D + e0) + lr);
+        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hw));
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        hts[2 * lr] = h.x;
+        hts[2 * lr + 1] = h.y;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
       }
       // s H_i^T = s H_total^T + G_i at the tile's positions
       bool ok = mbar_wait(tfull + acc, (i >> 1) & 1, abort_flag, a.status, a.budget_ns);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (!ok) break;
-      const uint4* ht = reinterpret_cast<const uint4*>(a.htile + (size_t)bh * D * D + e0);
       // kept in L2 for the epilogue, which reads every image once right after this kernel
       const uint64_t keep = l2_policy_evict_last();
       // 64 positions at a time: each lane converts its row's 128 bytes into the warp's
@@ -228,9 +251,6 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
       uint8_t* stg = base + C::OFF_STG + (qd * 32) * 128;
 #pragma unroll 1
       for (int c64 = 0; c64 < HS_BN / 64; ++c64) {
-        uint4 hv[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) hv[k] = __ldg(ht + c64 * 8 + k);   // the same 16 bytes for every lane
         uint32_t v[64];
         tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + c64 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
         tmem_ld32(tmem + lane_base + (uint32_t)(acc * HS_BN + c64 * 64 + 32),
@@ -239,13 +259,13 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
         __syncwarp();   // the previous chunk's staging rows have been read
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint32_t hu[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+          const float4 h0 = *reinterpret_cast<const float4*>(hts + c64 * 64 + k * 8);       // same for every lane
+          const float4 h1 = *reinterpret_cast<const float4*>(hts + c64 * 64 + k * 8 + 4);
+          const float h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
           uint32_t o[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hu[u]));
-            o[u] = h2u(h.x + __uint_as_float(v[k * 8 + 2 * u]), h.y + __uint_as_float(v[k * 8 + 2 * u + 1]));
-          }
+          for (int u = 0; u < 4; ++u)
+            o[u] = h2u(h[2 * u] + __uint_as_float(v[k * 8 + 2 * u]), h[2 * u + 1] + __uint_as_float(v[k * 8 + 2 * u + 1]));
           *reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         __syncwarp();
@@ -272,17 +292,17 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
 
 }  // namespace
 
-cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const HselArgs& a,
-                        cudaStream_t st) {
+cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const CUtensorMap& tz,
+                        const HselArgs& a, cudaStream_t st) {
   constexpr int kSMs = 148;   // B200 streaming multiprocessors
-  const int tiles = s.BH * ((s.d * s.d) / HS_BN) * ((s.nq + HS_BM - 1) / HS_BM);
+  const int tiles = s.BH * ((s.d * s.d) / HS_BN + 1) * ((s.nq + HS_BM - 1) / HS_BM);
   const int grid = tiles < kSMs ? tiles : kSMs;
   if (s.d == 128) {
     cudaFuncSetAttribute(hsel_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, HsCfg::SMEM);
-    hsel_kernel<128><<<grid, HS_THREADS, HsCfg::SMEM, st>>>(tmask, timg, s, a);
+    hsel_kernel<128><<<grid, HS_THREADS, HsCfg::SMEM, st>>>(tmask, timg, tz, s, a);
   } else {
     cudaFuncSetAttribute(hsel_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, HsCfg::SMEM);
-    hsel_kernel<64><<<grid, HS_THREADS, HsCfg::SMEM, st>>>(tmask, timg, s, a);
+    hsel_kernel<64><<<grid, HS_THREADS, HsCfg::SMEM, st>>>(tmask, timg, tz, s, a);
   }
   return cudaGetLastError();
 }

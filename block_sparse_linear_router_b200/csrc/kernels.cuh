@@ -82,7 +82,8 @@ cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, co
 // H_total^T / Z_total (fp32) from the chunk partials; optionally (vamax given)
 // the fp16 image of s H_total^T in the h_mode-2 layout and s per head.
 cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, const unsigned* vamax,
-                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st);
+                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st,
+                                 const float* z = nullptr, uint16_t* z16 = nullptr);
 
 // ---- sparse branch (sparse.cu) --------------------------------------------
 struct SparseArgs {
@@ -104,22 +105,21 @@ size_t sparse_smem_bytes(int d, int quant);
 struct HselArgs {
   const uint16_t* htile;  // fp16 s H_total^T operand images [BH][d*d]
   const float* Ztot;      // [BH][d] Z_total
-  const float* z;         // [BH][nk][d] z_j
-  const int32_t* idx;     // [BH][nq][k]
   uint16_t* hi;           // out: fp16 s H_i^T operand images [BH][nq][d*d]
   float* Zi;              // out: [BH][nq][d] Z_i
   unsigned* status;
   unsigned long long budget_ns;
 };
 // tmask: the fp16 mask [BH*nq][nk8], box {64, 128}; timg: the -s h_j^T images as a
-// [BH*nk][d*d] fp16 matrix, box {64, 64}; both with 128-byte swizzle.
-cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const HselArgs& a,
-                        cudaStream_t st);
+// [BH*nk][d*d] fp16 matrix, box {64, 64}; tz: the fp16 z_j as a [BH*nk][d] matrix,
+// box {64, 64}; all with 128-byte swizzle.
+cudaError_t launch_hsel(const Shape& s, const CUtensorMap& tmask, const CUtensorMap& timg, const CUtensorMap& tz,
+                        const HselArgs& a, cudaStream_t st);
 
 struct EpilogueArgs {
   const void* q;          // bf16 [BH][N][d]
   const uint16_t* hi;     // fp16 s H_i^T operand images [BH][nq][d*d]
-  const float* Zi;        // [BH][nq][d]
+  const float* Zi;        // [BH][nq][d] Z_i
   const float* hscale;    // [BH] s
   const void* os;         // [BH][N][d] O_s: fp32, or fp16 O_s / s_v when os_half
   int os_half;

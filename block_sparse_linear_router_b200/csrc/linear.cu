@@ -480,7 +480,8 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
 __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const float* __restrict__ zpart, int G, int D,
                                      int N, const unsigned* __restrict__ vamax, float* __restrict__ Htot,
                                      float* __restrict__ Ztot, uint16_t* __restrict__ htile,
-                                     float* __restrict__ hscale) {
+                                     float* __restrict__ hscale, const float* __restrict__ z,
+                                     uint16_t* __restrict__ z16, int nk) {
   __shared__ float red[8];
   const int bh = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -515,6 +516,9 @@ __global__ void linear_reduce_kernel(const float* __restrict__ hpart, const floa
     for (int g = 0; g < G; ++g) s += __ldg(zpart + ((size_t)bh * G + g) * D + threadIdx.x);
     Ztot[(size_t)bh * D + threadIdx.x] = s;
   }
+  if (z16)   // z_j as fp16, the operand of the selected-state product
+    for (int x = e; x < nk * D; x += DD)
+      z16[(size_t)bh * nk * D + x] = __half_as_ushort(__float2half_rn(__ldg(z + (size_t)bh * nk * D + x)));
 }
 
 constexpr int kSMs = 148;   // B200 streaming multiprocessors
@@ -548,11 +552,12 @@ cudaError_t launch_linear_state(const Shape& s, const void* k, const void* v, co
 }
 
 cudaError_t launch_linear_reduce(const Shape& s, const float* hpart, const float* zpart, const unsigned* vamax,
-                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st) {
+                                 float* Htot, float* Ztot, uint16_t* htile, float* hscale, cudaStream_t st,
+                                 const float* z, uint16_t* z16) {
   const int DD = s.d * s.d;
   dim3 grid((DD + 255) / 256, s.BH);
   linear_reduce_kernel<<<grid, 256, 0, st>>>(hpart, zpart, s.G, s.d, s.N, vamax, Htot, Ztot,
-                                             htile, hscale);
+                                             htile, hscale, z, z16, s.nk);
   return cudaGetLastError();
 }
 
