@@ -119,12 +119,14 @@ def work_model(w, k):
 # kernel source they were taken on: sha256 prefix of the stage's kernel file(s) ("a.cu+b.cu")
 # + device.cuh + kernels.cuh.
 MEASURED_TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum, --set full capture
-    "sparse": ("sparse.cu", "3a73ccef7b0d189c", 298.1e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
-    # dram__bytes.sum.per_second x gpu__time_duration.sum, section captures
-    "epilogue": ("epilogue.cu", "1b0cc1424c18eeed", 596.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "linear_state": ("linear.cu", "67c76cddfc1bdc85", 471.3e6, "ncu dram__bytes.sum.per_second x duration"),
-    "router": ("router.cu", "4eadfd52602acf06", 345.5e6, "ncu dram__bytes.sum.per_second x duration (pool_kernel)"),
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch (one forward's launches for a
+    # stage of several kernels), section captures of the bench command (profiles/)
+    "sparse": ("sparse.cu", "1509063481d9cb60", 214.7e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    "epilogue": ("hsel.cu+epilogue.cu", "6ff15388867ce7de", 646.0e6,
+                 "ncu dram__bytes_read.sum + dram__bytes_write.sum (hsel_kernel + epilogue_kernel)"),
+    "linear_state": ("linear.cu", "853563ed08f4b842", 471.7e6,
+                     "ncu dram__bytes_read.sum + dram__bytes_write.sum (linear_state_kernel)"),
+    "router": ("router.cu", "a63d2887061c43d4", 345.3e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum (pool_kernel)"),
 }
 
 
