@@ -380,11 +380,17 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
   // exports fp32 O_s), else fp32 (written straight into the export when there is one)
   void* os = (!quant && desc->dbg_os) ? static_cast<void*>(desc->dbg_os) : at<void>(desc, L.os);
   SparseArgs sa{idx, at<float>(desc, L.sq), at<float>(desc, L.sk), at<float>(desc, L.sv), os, desc->status, g_budget_ns};
+  // the selected-state product does not depend on the sparse branch: it goes on the
+  // auxiliary stream, enqueued after the sparse kernel, and takes the SMs that the
+  // sparse branch's last CTAs leave
+  const bool hsel_on = s.k < s.nk;
+  if (hsel_on) SLA2_TRY(cudaEventRecord(aux->fork, st));
   SLA2_TRY(launch_sparse(s, quant, tq, tk, tv, sa, st));
   SLA2_TRY(mark(3));
 
   // the linear branch's s H_i^T and Z_i for every query block (one product with the mask)
-  if (s.k < s.nk) {
+  if (hsel_on) {
+    SLA2_TRY(cudaStreamWaitEvent(aux->stream, aux->fork, 0));
     CUtensorMap tm, ti, tz;
     const uint64_t nk8 = ((uint64_t)s.nk + 7) & ~uint64_t(7);
     if (!make_map(&tm, mask16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, nk8, (uint64_t)s.BH * s.nq, 64, 128,
@@ -401,7 +407,9 @@ sla2_status forward_body(const sla2_desc* desc, const Shape& s, int H, const Lay
     ha.Zi = at<float>(desc, L.Zi);
     ha.status = desc->status;
     ha.budget_ns = g_budget_ns;
-    SLA2_TRY(launch_hsel(s, tm, ti, tz, ha, st));
+    SLA2_TRY(launch_hsel(s, tm, ti, tz, ha, aux->stream));
+    SLA2_TRY(cudaEventRecord(aux->join, aux->stream));
+    SLA2_TRY(cudaStreamWaitEvent(st, aux->join, 0));
   }
 
   EpilogueArgs ea{};

@@ -181,8 +181,10 @@ sla2_status sla2_linear_state(const sla2_desc* desc, const void* k, const void* 
  * All intermediates live in desc->workspace; optional debug exports in desc.
  * The linear-state pass runs on a library-owned non-blocking stream, forked
  * from and joined back into `stream` with events, concurrently with the
- * router's projections, logits and top-k on `stream`. That stream and its two events are
- * created by the first call on each device and kept until the process exits;
+ * router's projections, logits and top-k on `stream`; the selected-state product
+ * (H_i, Z_i of every query block) runs on it too, beside the sparse branch. That
+ * stream and its two events are created by the first call on each device and
+ * kept until the process exits;
  * make that first call outside any stream capture. Later calls can be captured
  * (the fork and join become graph edges). Calls from several host threads are
  * serialised while they enqueue.
