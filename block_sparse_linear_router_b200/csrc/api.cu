@@ -54,8 +54,8 @@ sla2_status check_desc(const sla2_desc* d, float frac, Shape* s) {
 
 // Workspace regions (each 256-byte aligned).
 struct Layout {
-  size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, mask16, qhat, sq, vamax, khat, sk, vhatT, sv, h, z, hpart,
-      zpart, Htot, Ztot, htile, hscale, hi, Zi, z16, os, total;
+  size_t qbar, ksum, c64, c32, kbs, A, Bk, scores, mask, idx, mask16, qhat, sq, vamax, csum, khat, sk, vhatT, sv, h, z,
+      hpart, zpart, Htot, Ztot, htile, hscale, hi, Zi, z16, os, total;
 };
 
 Layout make_layout(const Shape& s, int quant) {
@@ -82,6 +82,7 @@ Layout make_layout(const Shape& s, int quant) {
   L.qhat = take(quant ? BH * N * d : 0);
   L.sq = take(BH * nq * 4);
   L.vamax = take(BH * d * 4);
+  L.csum = take(BH * d * 8);         // fp64 column sums of K (pool pass, atomic adds)
   L.khat = take(quant ? BH * N * d : 0);
   L.sk = take(BH * nk * 4);
   L.vhatT = take(BH * nk * d * BKB * (quant ? 1 : 2));
@@ -131,6 +132,7 @@ BwdLayout make_bwd_layout(const Shape& s) {
   L.idx = take(BH * nq * k * 4);
   L.sq = take(BH * nq * 4);
   L.vamax = take(BH * d * 4);
+  L.csum = take(BH * d * 8);
   L.h = take(BH * nk * d * d * 4);
   L.z = take(BH * nk * d * 4);
   L.hpart = take(BH * G * d * d * 4);
@@ -203,13 +205,17 @@ sla2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA2_OK : SLA
 // Router, first part: the pass over Q, K (and V) and the column means.
 sla2_status router_head(const sla2_desc* d, const Shape& s, const Layout& L, const void* q, const void* k,
                         const void* v, int quant, cudaStream_t st) {
-  // with V given, its per-channel |V| max (V-hat scales, fp16 scale of the linear state)
-  if (v) SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, (size_t)s.BH * s.d * 4, st));
+  // the column sums start at zero; with V given, so does its per-channel |V| max (V-hat
+  // scales, fp16 scale of the linear state), which sits right before them
+  if (v)
+    SLA2_TRY(cudaMemsetAsync(at<void>(d, L.vamax), 0, L.csum - L.vamax + (size_t)s.BH * s.d * 8, st));
+  else
+    SLA2_TRY(cudaMemsetAsync(at<void>(d, L.csum), 0, (size_t)s.BH * s.d * 8, st));
   SLA2_TRY(launch_pool(s, q, k, v, at<float>(d, L.qbar), at<double>(d, L.ksum),
                        quant ? at<int8_t>(d, L.qhat) : nullptr, at<float>(d, L.sq),
-                       v ? at<unsigned>(d, L.vamax) : nullptr, d->status, g_budget_ns, st));
+                       v ? at<unsigned>(d, L.vamax) : nullptr, d->status, g_budget_ns, st, at<double>(d, L.csum)));
   SLA2_TRY(launch_colmean(s, at<double>(d, L.ksum), at<double>(d, L.c64), at<float>(d, L.c32), at<float>(d, L.kbs),
-                           st));
+                           st, at<double>(d, L.csum)));
   return SLA2_OK;
 }
 

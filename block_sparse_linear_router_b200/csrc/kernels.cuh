@@ -26,16 +26,19 @@ struct Shape {
 // Pass over Q, K (and V): pooled Q (fp32), exact fp64 column sums per key block,
 // optional INT8 Q-hat + s_q, optional per-channel |V| max (atomic, as uint bits).
 // Its pipeline waits are bounded by budget_ns (status gets the timeout code).
+// csum (optional, zero at launch): the head's fp64 column sums of K, gathered with
+// atomic adds (exact sums, so independent of their order).
 cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void* v, float* qbar, double* ksum,
                         int8_t* qhat, float* sq, unsigned* vamax, unsigned* status, unsigned long long budget_ns,
-                        cudaStream_t st);
+                        cudaStream_t st, double* csum = nullptr);
 constexpr unsigned long long kDefaultWaitBudgetNs = 2000000000ull;   // 2 s per device wait
 // The budget every bounded device wait of the next launches gets (the default, or the
 // value last set by sla2_set_wait_budget_ns); implemented in api.cu.
 unsigned long long wait_budget_ns();
-// colmean (fp64 and fp32) from the per-block sums, and the smoothed pooled keys.
+// colmean (fp64 and fp32) from the per-block sums (or, given csum, from the column
+// sums the pool pass gathered), and the smoothed pooled keys.
 cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, float* kbar_s,
-                           cudaStream_t st);
+                           cudaStream_t st, const double* csum = nullptr);
 // A = Qbar Wq, Bk = (Kbar - c) Wk, fp32.
 cudaError_t launch_proj(const Shape& s, int H, const float* qbar, const float* kbar_s, const float* wq,
                         const float* wk, float* A, float* Bk, cudaStream_t st);

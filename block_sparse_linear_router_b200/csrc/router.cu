@@ -77,7 +77,8 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat
                                                                int nq, int nk, float* __restrict__ qbar,
                                                                double* __restrict__ ksum, int8_t* __restrict__ qhat,
                                                                float* __restrict__ sq, unsigned* __restrict__ vamax,
-                                                               unsigned* status, unsigned long long budget_ns) {
+                                                               unsigned* status, unsigned long long budget_ns,
+                                                               double* __restrict__ csum) {
   using C = PoolCfg<D>;
   constexpr int TPR = C::TPR, RPP = C::RPP, NP = C::NP, NS = C::NS;
   extern __shared__ __align__(128) uint8_t pool_smem[];
@@ -203,6 +204,10 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat
       qbar[((size_t)bh * nq + i) * D + tid] = (float)(sqs / (double)BQ);
       ksum[((size_t)bh * nk + 2 * i) * D + tid] = s0;
       ksum[((size_t)bh * nk + 2 * i + 1) * D + tid] = s1;
+      if (csum) {   // the head's column sums: exact fp64 sums, so the order of the adds does not matter
+        atomicAdd(csum + (size_t)bh * D + tid, s0);
+        atomicAdd(csum + (size_t)bh * D + tid, s1);
+      }
       if (v) atomicMax(vamax + (size_t)bh * D + tid, __float_as_uint(m));   // non-negative floats order like their bits
     }
     // ---- INT8 Q-hat with the block's |Q| maximum
@@ -264,6 +269,24 @@ __global__ void __launch_bounds__(256) colmean_kbar_kernel(const double* __restr
     const size_t o = ((size_t)bh * nk + j) * D + col;
     kbar_s[o] = (float)(ksum[o] / (double)BKB - m);
   }
+}
+
+// The same from the head's column sums gathered by the pool pass: one thread per
+// (head, key block, column), c = csum / N in fp64 and Kbar_j - c in fp32.
+__global__ void __launch_bounds__(256) kbar_kernel(const double* __restrict__ csum, const double* __restrict__ ksum,
+                                                   int BH, int nk, int N, int D, double* __restrict__ c64,
+                                                   float* __restrict__ c32, float* __restrict__ kbar_s) {
+  const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (size_t)BH * nk * D) return;
+  const int col = (int)(e % D);
+  const size_t bhj = e / D;
+  const int bh = (int)(bhj / nk), j = (int)(bhj % nk);
+  const double m = csum[(size_t)bh * D + col] / (double)N;
+  if (j == 0) {
+    c64[(size_t)bh * D + col] = m;
+    c32[(size_t)bh * D + col] = (float)m;
+  }
+  kbar_s[e] = (float)(ksum[e] / (double)BKB - m);
 }
 
 // Batched fp32 SIMT GEMM for the router's projections, both of them in one
@@ -595,7 +618,7 @@ cudaError_t launch_soft_topk(const Shape& s, const float* scores, float tau, flo
 
 cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void* v, float* qbar, double* ksum,
                         int8_t* qhat, float* sq, unsigned* vamax, unsigned* status, unsigned long long budget_ns,
-                        cudaStream_t st) {
+                        cudaStream_t st, double* csum) {
   constexpr int kSMs = 148;   // B200 streaming multiprocessors
   const int items = s.BH * s.nq;
   const int grid = items < kSMs ? items : kSMs;
@@ -605,18 +628,23 @@ cudaError_t launch_pool(const Shape& s, const void* q, const void* k, const void
   if (s.d == 128) {
     cudaFuncSetAttribute(pool_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, PoolCfg<128>::SMEM);
     pool_kernel<128><<<grid, POOL_THREADS, PoolCfg<128>::SMEM, st>>>(qb, kb, vb, s.BH, s.N, s.nq, s.nk, qbar, ksum,
-                                                                      qhat, sq, vamax, status, budget_ns);
+                                                                      qhat, sq, vamax, status, budget_ns, csum);
   } else {
     cudaFuncSetAttribute(pool_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, PoolCfg<64>::SMEM);
     pool_kernel<64><<<grid, POOL_THREADS, PoolCfg<64>::SMEM, st>>>(qb, kb, vb, s.BH, s.N, s.nq, s.nk, qbar, ksum,
-                                                                    qhat, sq, vamax, status, budget_ns);
+                                                                    qhat, sq, vamax, status, budget_ns, csum);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_colmean(const Shape& s, const double* ksum, double* c64, float* c32, float* kbar_s,
-                           cudaStream_t st) {
-  colmean_kbar_kernel<<<dim3(s.BH, s.d / 32), 256, 0, st>>>(ksum, s.nk, s.N, s.d, c64, c32, kbar_s);
+                           cudaStream_t st, const double* csum) {
+  if (csum) {
+    const size_t n = (size_t)s.BH * s.nk * s.d;
+    kbar_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(csum, ksum, s.BH, s.nk, s.N, s.d, c64, c32, kbar_s);
+  } else {
+    colmean_kbar_kernel<<<dim3(s.BH, s.d / 32), 256, 0, st>>>(ksum, s.nk, s.N, s.d, c64, c32, kbar_s);
+  }
   return cudaGetLastError();
 }
 

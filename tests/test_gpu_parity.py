@@ -251,11 +251,13 @@ def test_bounded_wait_reports_timeout_and_context_survives(sla2):
     assert int(status.item()) == 0
 
 
-@pytest.mark.parametrize("shape", [(1, 3, 8192, 128, 0.03), (1, 3, 8192, 64, 0.1), (1, 3, 8192, 128, 0.001)])
+@pytest.mark.parametrize("shape", [(1, 3, 8192, 128, 0.03), (1, 3, 8192, 64, 0.1), (1, 3, 8192, 128, 0.001),
+                                   (1, 8, 8192, 128, 0.03)])
 def test_more_query_blocks_than_sms(sla2, shape):
-    """192 (head, query block) items: the persistent kernels walk several items
-    per CTA (k = 1, 3 and 12 key blocks per item) and the linear-state pass
-    splits heads into chunks."""
+    """192 or 512 (head, query block) items: the persistent kernels walk several
+    items per CTA (k = 1, 3 and 12 key blocks per item; up to four items, so that
+    the epilogue's two-slot rings are each reused) and the linear-state pass splits
+    heads into chunks."""
     B, H, N, d, frac = shape
     _compare_full(sla2, make_custom(B, H, N, d, frac, seed=32), frac, f"multiwave-d{d}")
 
