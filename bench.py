@@ -121,12 +121,12 @@ def work_model(w, k):
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (one forward's launches for a
     # stage of several kernels), section captures of the bench command (profiles/)
-    "sparse": ("sparse.cu", "1509063481d9cb60", 214.7e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
-    "epilogue": ("hsel.cu+epilogue.cu", "6ff15388867ce7de", 646.0e6,
+    "sparse": ("sparse.cu", "10a687aab6afa0d9", 214.0e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    "epilogue": ("hsel.cu+epilogue.cu", "e75c302ceb107816", 646.8e6,
                  "ncu dram__bytes_read.sum + dram__bytes_write.sum (hsel_kernel + epilogue_kernel)"),
-    "linear_state": ("linear.cu", "853563ed08f4b842", 471.7e6,
+    "linear_state": ("linear.cu", "aa99c2dfd7748bf6", 471.5e6,
                      "ncu dram__bytes_read.sum + dram__bytes_write.sum (linear_state_kernel)"),
-    "router": ("router.cu", "a63d2887061c43d4", 345.3e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum (pool_kernel)"),
+    "router": ("router.cu", "c883e40e8855ada8", 345.7e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum (pool_kernel)"),
 }
 
 

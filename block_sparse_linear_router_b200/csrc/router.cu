@@ -128,6 +128,11 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat
 
   // -------------------------------------------------------------------- consumers
   const int cg = tid % TPR, rg = tid / TPR;   // channels cg*4 .. +3; rows rg, rg + RPP, ...
+  // the head's column sums (threads tid < D): this CTA's block sums of the current head,
+  // added to csum when the head changes (exact fp64 sums, so neither the grouping nor
+  // the order of the adds changes the result)
+  double run = 0.0;
+  int run_bh = -1;
   int n = 0;
   for (int it = blockIdx.x; it < items; it += gridDim.x, ++n) {
     const int s = n % NS;
@@ -204,9 +209,14 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat
       qbar[((size_t)bh * nq + i) * D + tid] = (float)(sqs / (double)BQ);
       ksum[((size_t)bh * nk + 2 * i) * D + tid] = s0;
       ksum[((size_t)bh * nk + 2 * i + 1) * D + tid] = s1;
-      if (csum) {   // the head's column sums: exact fp64 sums, so the order of the adds does not matter
-        atomicAdd(csum + (size_t)bh * D + tid, s0);
-        atomicAdd(csum + (size_t)bh * D + tid, s1);
+      if (csum) {
+        if (bh != run_bh) {
+          if (run_bh >= 0) atomicAdd(csum + (size_t)run_bh * D + tid, run);
+          run = 0.0;
+          run_bh = bh;
+        }
+        run += s0;
+        run += s1;
       }
       if (v) atomicMax(vamax + (size_t)bh * D + tid, __float_as_uint(m));   // non-negative floats order like their bits
     }
@@ -239,6 +249,7 @@ __global__ void __launch_bounds__(POOL_THREADS, 1) pool_kernel(const __nv_bfloat
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + s);
   }
+  if (csum && tid < D && run_bh >= 0) atomicAdd(csum + (size_t)run_bh * D + tid, run);
 }
 
 // c = (sum of the exact per-block column sums) / N in fp64, then the smoothed
