@@ -11,8 +11,9 @@
 // items (g counts key blocks over all items of the CTA). 192 threads:
 //   warps 0-3  softmax: thread t owns query row t (= TMEM lane t); online
 //              softmax with one running-max update per key block; P written
-//              to shared memory as e4m3 (x448 fixed scale) or bf16; O rescaled
-//              in TMEM when a row max grows; at the end of an item the row is
+//              as e4m3 (x448 fixed scale) into TMEM, over key columns 0-15 of
+//              its own S buffer, or as bf16 to shared memory; O rescaled in
+//              TMEM when a row max grows; at the end of an item the row is
 //              normalised and stored while the next item's S is computed (fp32
 //              O_s, or on the quantised path the fp16 row O_s / s_v: a
 //              weighted mean of e4m3 V-hat codes, so |.| <= 448 and the
@@ -22,10 +23,13 @@
 //              rings of NS stages (no multicast): a K stage is released when
 //              its QK has finished, a V stage when its PV has, and V is loaded
 //              one block behind K because PV runs two blocks behind QK.
-//   warp 5     tcgen05 issuer, in the order QK(g), PV(g-2): S_g = Q K_j^T into
-//              one of two TMEM buffers (kind::i8 -> s32, or kind::f16 -> f32)
-//              as soon as that buffer's previous S has been read, and
-//              O += P_g V_j (kind::f8f6f4 e4m3 or kind::f16 bf16 -> f32).
+//   warp 5     tcgen05 issuer, in the order PV(g-2), QK(g): O += P_g V_j
+//              (kind::f8f6f4 e4m3 with P from TMEM, or kind::f16 bf16 -> f32),
+//              and S_g = Q K_j^T into one of two TMEM buffers (kind::i8 -> s32,
+//              or kind::f16 -> f32) as soon as that buffer's previous S has been
+//              read. The tensor pipe
+//              runs MMAs in issue order, so QK(g) overwrites P(g-2) only after
+//              PV(g-2) has read it.
 // TMEM columns: [0,64) S buffer 0, [64,128) S buffer 1, [128,128+D) O.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -36,6 +40,16 @@
 namespace sla2 {
 
 namespace {
+
+// D[tmem] (+)= A[tmem] x B[smem]^T for e4m3 operands: A (M = 128 lanes, four 8-bit K
+// values per 32-bit column) read from tensor memory, B by descriptor.
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 
 template <int D, bool QUANT>
 struct Cfg {
@@ -59,7 +73,7 @@ struct Cfg {
   static constexpr int OFF_K = 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * K_BYTES;
   static constexpr int OFF_P = OFF_V + NS * V_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_P + (QUANT ? 0 : 2 * P_BYTES);   // the INT8 path keeps P in TMEM
   // barriers: q_full[2], q_free[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS],
   //           s_full[2], s_empty[2], p_full[2], p_free[2], o_full, o_free, drain
   static constexpr int NBAR = 4 + 4 * NS + 8 + 3;
@@ -69,6 +83,7 @@ struct Cfg {
   static_assert(SMEM <= 232448, "dynamic shared memory per CTA (227 KB)");
   static_assert(!QUANT || 2 * (SMEM + 1024) <= 233472, "two CTAs per SM (228 KB, 1 KB reserved per CTA)");
   static constexpr uint32_t IDESC_QK = QUANT ? make_idesc(2, 1, 1, 128, 64) : make_idesc(1, 1, 1, 128, 64);
+
   static constexpr uint32_t IDESC_PV = QUANT ? make_idesc(1, 0, 0, 128, D) : make_idesc(1, 1, 1, 128, D);
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t COL_O = 128;
@@ -267,12 +282,12 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
         const uint32_t pt = p_addr + b * C::P_BYTES, vt = v_addr + st * C::V_BYTES;
 #pragma unroll
         for (int ks = 0; ks < C::PV_STEPS; ++ks) {
-          const uint64_t ad = make_sdesc(pt + ks * 32, 8 * C::VP_ROW, C::VP_LAYOUT);
           const uint64_t bd = make_sdesc(vt + ks * 32, 8 * C::VP_ROW, C::VP_LAYOUT);
-          if (QUANT)
-            mma_f8(tmem + C::COL_O, ad, bd, C::IDESC_PV, (n > 0 || ks > 0));
+          if (QUANT)   // P(g) in TMEM columns b*64 .. +15, 8 columns per 32-value K step
+            mma_f8_ts(tmem + C::COL_O, tmem + b * 64 + ks * 8, bd, C::IDESC_PV, (n > 0 || ks > 0));
           else
-            mma_f16(tmem + C::COL_O, ad, bd, C::IDESC_PV, (n > 0 || ks > 0));
+            mma_f16(tmem + C::COL_O, make_sdesc(pt + ks * 32, 8 * C::VP_ROW, C::VP_LAYOUT), bd, C::IDESC_PV,
+                    (n > 0 || ks > 0));
         }
         tc_commit(v_empty + st);
         tc_commit(p_free + b);
@@ -280,9 +295,11 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
         return true;
       };
       bool ok = true;
+      // PV(g - 2) goes into the tensor pipe ahead of QK(g): on the INT8 path QK(g) overwrites
+      // the TMEM columns that hold P(g - 2), and the pipe runs MMAs in issue order
       for (int g = 0; ok && g < nblocks + 2; ++g) {
-        if (g < nblocks) ok = issue_qk(g);
-        if (ok && g >= 2) ok = issue_pv(g - 2);
+        if (g >= 2) ok = issue_pv(g - 2);
+        if (ok && g < nblocks) ok = issue_qk(g);
       }
       if (!ok) {
         // wait for every MMA issued so far before the tensor memory is released
@@ -332,7 +349,8 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
         // Raw logits as fp32 pairs. For INT8 the s32 accumulator plus 0x4B400000 is
         // the bit pattern of 12582912 + S exactly (|S| < 2^22); subtracting
         // 12582912 is exact too, so S becomes a float without an int->float
-        // conversion.
+        // conversion. (Presetting the accumulator to 0x4B400000 would save the adds,
+        // but key columns 0-15 hold P(g - 2) until QK(g) overwrites them.)
         uint64_t f2[32];
         const uint64_t off2 = f2_pack(-12582912.f, -12582912.f);
 #pragma unroll
@@ -388,20 +406,19 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
         f2_unpack(f2_add(rs2a, rs2b), ra0, ra1);
         l = l * corr + (ra0 + ra1);
         m = m_new;
-        // P buffer b was last read by PV g-2
+        // P buffer b was last read by PV g-2 (on the INT8 path QK(g) has already followed
+        // PV(g-2) in the tensor pipe; the wait keeps this warp's view of the p_free phases
+        // in step for the rescale's wait below)
         if (g >= 2) {
           ok = mbar_wait(p_free + b, ((g >> 1) - 1) & 1, abortf, a.status, a.budget_ns);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
-        uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
         if (QUANT) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int pc = ch ^ ((r >> 1) & 3);        // 64-byte swizzle
-            *reinterpret_cast<uint4*>(prow + pc * 16) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          }
+          // e4m3 P(g) into key columns 0-15 of its own S buffer (S(g) is in registers), four
+          // values per column: the A operand of PV(g)
+          tmem_st16(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[16]>(pk));
         } else {
+          uint8_t* prow = sP + b * C::P_BYTES + r * C::VP_ROW;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const int pc = ch ^ (r & 7);               // 128-byte swizzle
@@ -409,7 +426,7 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
                 make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
           }
         }
-        fence_proxy_async_smem();
+        if (!QUANT) fence_proxy_async_smem();
         // O must be rescaled by corr (after PV n-1 has finished) before PV n adds to it;
         // P is already stored, so its write and proxy fence overlap this wait
         if (n >= 1 && __any_sync(0xffffffffu, corr != 1.f)) {
@@ -453,6 +470,7 @@ __global__ void __launch_bounds__(192, QUANT ? 2 : 1) sparse_kernel(const __grid
           }
           tmem_wait_st();
         }
+        if (QUANT) tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full + b);     // P written and O rescaled
