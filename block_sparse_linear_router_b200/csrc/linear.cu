@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
           amax = fmaxf(amax, fabsf(x[u][c]));
         }
       }
+      float ablk = INFINITY;         // the block's max |K_s| (quantised path)
       if (o.khat) {
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
         conv_sync();
         const float a = fmaxf(fmaxf(fmaxf(ared[0], ared[1]), fmaxf(ared[2], ared[3])),
                               fmaxf(fmaxf(ared[4], ared[5]), fmaxf(ared[6], ared[7])));
+        ablk = a;
         const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
         const bool magic = __float_as_uint(inv) < 0x7F800000u;   // finite (block-uniform); else the saturating path
 #pragma unroll
@@ -357,13 +359,20 @@ __global__ void __launch_bounds__(LIN_THREADS, 2) linear_state_kernel(const __gr
       float zc[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) zc[c] = 0.f;
+      // phi is a softmax over the features, so any shift works: with the block's max |K_s|
+      // (a bound on every token's max) known, exp(x - a) >= 2^-116 for a < 40 and the
+      // per-token max (four shuffle levels a token) is not needed; else the token's own max
+      const bool shift_blk = ablk < 40.f;   // block-uniform
 #pragma unroll
       for (int u = 0; u < TPT; ++u) {
-        float m = x[u][0];
+        float m = ablk;
+        if (!shift_blk) {
+          m = x[u][0];
 #pragma unroll
-        for (int c = 1; c < 8; ++c) m = fmaxf(m, x[u][c]);
+          for (int c = 1; c < 8; ++c) m = fmaxf(m, x[u][c]);
 #pragma unroll
-        for (int off = EG / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          for (int off = EG / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        }
         // exp(x - m) as 2^(x log2 e - m log2 e); phi is rounded to fp16 for the MMA
         const float mb = m * 1.4426950408889634f;
         float sum = 0.f;
