@@ -121,10 +121,10 @@ def work_model(w, k):
 MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (one forward's launches for a
     # stage of several kernels), section captures of the bench command (profiles/)
-    "sparse": ("sparse.cu", "10a687aab6afa0d9", 214.0e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
+    "sparse": ("sparse.cu", "24fb3fc0b54919cd", 213.6e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
     "epilogue": ("hsel.cu+epilogue.cu", "e75c302ceb107816", 646.8e6,
                  "ncu dram__bytes_read.sum + dram__bytes_write.sum (hsel_kernel + epilogue_kernel)"),
-    "linear_state": ("linear.cu", "aa99c2dfd7748bf6", 471.5e6,
+    "linear_state": ("linear.cu", "7af3af7e33104418", 470.9e6,
                      "ncu dram__bytes_read.sum + dram__bytes_write.sum (linear_state_kernel)"),
     "router": ("router.cu", "c883e40e8855ada8", 345.7e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum (pool_kernel)"),
 }
