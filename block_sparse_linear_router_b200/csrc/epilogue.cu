@@ -59,7 +59,8 @@ struct EpiCfg {
   static constexpr int NO = D == 128 ? 2 : 4;        // ring O slots (freed after the item's readout)
   static constexpr int OFF_O = NA * ASLOT;                    // ring O
   static constexpr int OFF_Z = OFF_O + NO * OSB;              // Z_i [NA][D]
-  static constexpr int OFF_XCH = OFF_Z + NA * D * 4;          // row max per half [2][BQ]
+  static constexpr int OFF_SV = OFF_Z + NA * D * 4;           // s_v of each ring O item's head [NO][D]
+  static constexpr int OFF_XCH = OFF_SV + NO * D * 4;         // row max per half [2][BQ]
   static constexpr int OFF_DEN = OFF_XCH + 2 * BQ * 4;        // denominator halves [2 buffers][2][BQ]
   static constexpr int OFF_BAR = OFF_DEN + 4 * BQ * 4;
   static constexpr int NBAR = 2 * NA + 2 * NO + 3;   // afull, afree [NA]; ofull, ofree [NO]; dfull [2]; drain
@@ -137,16 +138,18 @@ __device__ __forceinline__ void os_issue(const EpilogueArgs& a, size_t off, uint
 }
 
 // The chunk as fp32 O_s (fp16 O_s / s_v times s_v of columns col .. col + 15 of
-// head bh), also written to the fp32 export when there is one.
+// head bh, read from `svs`, the head's s_v row in shared memory, when given), also
+// written to the fp32 export when there is one.
 template <int D>
 __device__ __forceinline__ void os_convert(const EpilogueArgs& a, int bh, size_t off, int col, const OsChunk& c,
-                                           float (&o)[16]) {
+                                           float (&o)[16], const float* svs = nullptr) {
   if (a.os_half) {
     const float4* sv4 = reinterpret_cast<const float4*>(a.sv + (size_t)bh * D + col);
+    const float4* svs4 = reinterpret_cast<const float4*>(svs + col);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const uint32_t u[4] = {c.w[i].x, c.w[i].y, c.w[i].z, c.w[i].w};
-      const float4 s0 = __ldg(sv4 + 2 * i), s1 = __ldg(sv4 + 2 * i + 1);
+      const float4 s0 = svs ? svs4[2 * i] : __ldg(sv4 + 2 * i), s1 = svs ? svs4[2 * i + 1] : __ldg(sv4 + 2 * i + 1);
       const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -212,6 +215,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 1023) & ~uintptr_t(1023));
   // ring A slot b: s H_i^T image at b * ASLOT, Q rows at + TILE; ring O slot c at OFF_O + c * OSB
   float* zbuf = reinterpret_cast<float*>(base + C::OFF_Z);
+  float* svbuf = reinterpret_cast<float*>(base + C::OFF_SV);
   float* xch = reinterpret_cast<float*>(base + C::OFF_XCH);
   float* den_s = reinterpret_cast<float*>(base + C::OFF_DEN);
   uint64_t* afull = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);   // [NA] image, Q rows and Z_i landed
@@ -255,8 +259,8 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
     // ---------------------------------------------------------------- loader
     // lane 0, ring A: per item the s H_i^T image and the Z_i row (bulk copies) and the
     //   Q rows (TMA, 64-column slabs), once the MMA of item it - NA has completed;
-    // lane 1, ring O: per item the fp16 O_s rows (TMA; quantised path only), once the
-    //   readout of item it - NO is done.
+    // lane 1, ring O: per item the fp16 O_s rows (TMA; quantised path only) and the
+    //   head's s_v row (bulk copy), once the readout of item it - NO is done.
     if (lane < 2 && has_linear && (lane == 0 || a.os_half)) {
       const uint64_t once = l2_policy_evict_first();   // each is read once
       const int NR = lane == 0 ? C::NA : C::NO;
@@ -281,9 +285,12 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
           bulk_load(zbuf + sb * D, a.Zi + (size_t)w * D, (uint32_t)(D * 4), afull + sb);
         } else {
           uint8_t* slot = base + C::OFF_O + sb * C::OSB;
-          mbar_arrive_expect_tx(ofull + sb, (uint32_t)C::OSB);
+          mbar_arrive_expect_tx(ofull + sb, (uint32_t)(C::OSB + D * 4));
 #pragma unroll
           for (int sl = 0; sl < C::SLABS; ++sl) tma_load_2d(slot + sl * C::RSLAB, &tos, ofull + sb, sl * 64, row0);
+          // and the head's s_v row beside it (the readout's dequantisation scale, read
+          // from shared memory instead of 16 global loads a thread and item)
+          bulk_load(svbuf + sb * D, a.sv + (size_t)(w / s.nq) * D, (uint32_t)(D * 4), ofull + sb);
         }
       }
       if (!ok)   // copies in flight land before the CTA releases its shared memory
@@ -355,7 +362,7 @@ __global__ void __launch_bounds__(EPI_THREADS, 1) epilogue_kernel(const __grid_c
           tmem_ld16(tmem + lane_base + (uint32_t)(bp * D + col), v);
           tmem_wait_ld();
           float osv[16];
-          os_convert<D>(a, bh, off0 + cc * 16, col, ch[cc & 1], osv);
+          os_convert<D>(a, bh, off0 + cc * 16, col, ch[cc & 1], osv, a.os_half ? svbuf + so * D : nullptr);
           float ol[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) ol[c] = __uint_as_float(v[c]) * inv;
