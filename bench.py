@@ -122,7 +122,7 @@ MEASURED_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (one forward's launches for a
     # stage of several kernels), section captures of the bench command (profiles/)
     "sparse": ("sparse.cu", "24fb3fc0b54919cd", 213.6e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum"),
-    "epilogue": ("hsel.cu+epilogue.cu", "e75c302ceb107816", 646.8e6,
+    "epilogue": ("hsel.cu+epilogue.cu", "b529b50bf7bd5cde", 645.7e6,
                  "ncu dram__bytes_read.sum + dram__bytes_write.sum (hsel_kernel + epilogue_kernel)"),
     "linear_state": ("linear.cu", "7af3af7e33104418", 470.9e6,
                      "ncu dram__bytes_read.sum + dram__bytes_write.sum (linear_state_kernel)"),
