@@ -194,11 +194,23 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
     const int qd = warp & 3;                     // TMEM lane quadrant
     const int lr = qd * 32 + lane;               // accumulator row (query block within the tile)
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    // this thread's two s H_total^T positions of a tile (fp16 pair), loaded one tile ahead
+    // so that the L2 latency is not paid at the start of each tile
+    auto ht_load = [&](int t2) -> uint32_t {
+      if (t2 >= tiles) return 0u;
+      int bh2, m2, e2;
+      tile_of(t2, bh2, m2, e2);
+      if (e2 == (NT - 1) * HS_BN) return 0u;   // the z tile has none
+      return __ldg(reinterpret_cast<const uint32_t*>(a.htile + (size_t)bh2 * D * D + e2) + lr);
+    };
+    uint32_t hw_next = ht_load(blockIdx.x);
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       int bh, m0, e0;
       tile_of(t, bh, m0, e0);
       const int acc = i & 1;
+      const uint32_t hw = hw_next;
+      hw_next = ht_load(t + gridDim.x);
       if (e0 == (NT - 1) * HS_BN) {
         // the z tile: Z_i = Z_total - G_i, fp32, one query block per thread
         bool ok = mbar_wait(tfull + acc, (i >> 1) & 1, abort_flag, a.status, a.budget_ns);
@@ -227,11 +239,11 @@ __global__ void __launch_bounds__(HS_THREADS, 1) hsel_kernel(const __grid_consta
         mbar_arrive(tfree + acc);
         continue;
       }
-      // the tile's s H_total^T positions (fp32) into shared memory, two per thread; the
-      // previous tile's readers are past the barrier that ended it
+      // the tile's s H_total^T positions (fp32) into shared memory, two per thread (loaded
+      // during the previous tile); the previous tile's readers are past the barrier that
+      // ended it
       float* hts = reinterpret_cast<float*>(base + C::OFF_HT);
       {
-        const uint32_t hw = __ldg(reinterpret_cast<const uint32_t*>(a.htile + (size_t)bh * D * D + e0) + lr);
         const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hw));
         asm volatile("bar.sync 1, 128;" ::: "memory");
         hts[2 * lr] = h.x;
